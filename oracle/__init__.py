@@ -1,0 +1,24 @@
+"""CPU oracle for the sketched linear layer.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import or call anything in this package.
+The product path (the C-ABI library and its Python binding) never routes
+through it, and this package imports nothing from the product package.
+
+Everything here is plain, slow and written to be checked by eye against the
+definitions on the pages: "SpaLLM: Unified Compressive Adaptation of LLMs with
+Sketching" (section 2.2, Eq. 1 and groups per row; section 2.3, multiple LUT
+sets; section 2.4, the identity example) and the "Sketch to Adapt" OpenReview
+discussion (the corrected Eq. 6 and the mapping matrix M).  Floating point is
+float64 throughout; fp16 LUT values and bf16 activations widen exactly.
+
+Parity pins: every function here is pinned by a CPU test against something
+other than itself (a hand-derived golden fixture, a closed form, a library
+routine, an invariant, or finite differences).  No function is unpinned.
+"""
+from .sketch_oracle import (  # noqa: F401
+    row_stride_bytes, packed_bytes, pack, unpack, dequant, sketch_matrix,
+    dequant_via_sketch_matrix, forward, backward_input, backward_lut,
+    eq6_forward, eq6_backward_lut, bin_counts, trainable_params, lora_params,
+    compression_factor,
+)
