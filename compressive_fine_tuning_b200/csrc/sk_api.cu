@@ -1,0 +1,310 @@
+// C ABI of the sketched linear layer: argument validation and dispatch.
+//
+// Every entry point validates its arguments on the host before touching the
+// device, so a bad call returns a status without launching anything.  The
+// library allocates no device memory; the only device state is the check word
+// below, which kernels set when they meet data they cannot use (a task id out
+// of range, an index too large for its bit width).
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "sk_internal.cuh"
+
+namespace {
+
+__device__ unsigned int g_sk_check_word;
+
+thread_local std::string g_last_error;
+
+sk_status fail(sk_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+sk_status fail(sk_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+sk_status ok() { return SK_OK; }
+
+sk_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(SK_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr int kMaxDevices = 64;
+std::atomic<unsigned int*> g_check_ptr[kMaxDevices];
+std::atomic<int> g_device_ok[kMaxDevices];  // 0 unknown, 1 sm_100, -1 other
+
+// Current device's check word and capability (cached per device).
+sk_status device_state(unsigned int** check) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(SK_ERR_UNSUPPORTED, "device ordinal %d too large", dev);
+  int okv = g_device_ok[dev].load(std::memory_order_acquire);
+  if (okv == 0) {
+    int major = 0;
+    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    okv = (major == 10) ? 1 : -1;
+    g_device_ok[dev].store(okv, std::memory_order_release);
+  }
+  if (okv != 1) return fail(SK_ERR_UNSUPPORTED, "device %d is not sm_100 (B200); kernels are built for sm_100a only", dev);
+  unsigned int* p = g_check_ptr[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    e = cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_sk_check_word);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(check word)");
+    g_check_ptr[dev].store(p, std::memory_order_release);
+  }
+  *check = p;
+  return SK_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
+  if (a == nullptr || b == nullptr || an == 0 || bn == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + bn && b0 < a0 + an;
+}
+
+size_t row_bytes(int64_t d, int bits) {
+  if (bits < 2 || bits > 4 || d <= 0) return 0;
+  const int64_t raw = (d * bits + 7) / 8;
+  return (size_t)((raw + 15) / 16 * 16);
+}
+
+constexpr int64_t kMaxDim = int64_t(1) << 31;
+
+// Shape rules shared by the layer calls.
+sk_status check_shape(int bits, int gpr, int64_t n, int64_t d, int64_t T, int ntask) {
+  if (bits < 2 || bits > 4) return fail(SK_ERR_INVALID_ARG, "bits must be 2, 3 or 4 (got %d)", bits);
+  if (n < 1 || n % 8 != 0 || n >= kMaxDim) return fail(SK_ERR_INVALID_ARG, "n must be a positive multiple of 8 below 2^31 (got %lld)", (long long)n);
+  if (d < 32 || d % 32 != 0 || d >= kMaxDim) return fail(SK_ERR_INVALID_ARG, "d must be a positive multiple of 32 below 2^31 (got %lld)", (long long)d);
+  if (gpr < 1 || d % gpr != 0 || (d / gpr) % 32 != 0)
+    return fail(SK_ERR_INVALID_ARG, "gpr must divide d into groups whose size is a multiple of 32 (d=%lld, gpr=%d)", (long long)d, gpr);
+  if (T < 0 || T >= kMaxDim) return fail(SK_ERR_INVALID_ARG, "T must be in [0, 2^31) (got %lld)", (long long)T);
+  if (ntask < 1 || ntask > 65535) return fail(SK_ERR_INVALID_ARG, "ntask must be in [1, 65535] (got %d)", ntask);
+  return SK_OK;
+}
+
+sk::Problem make_problem(const void* packed, const uint16_t* lut, int bits, int gpr, int64_t n, int64_t d,
+                         int64_t T, const int32_t* task, int ntask, unsigned int* check) {
+  sk::Problem p;
+  p.packed = static_cast<const uint8_t*>(packed);
+  p.row_bytes = (int64_t)row_bytes(d, bits);
+  p.lut = lut;
+  p.bits = bits;
+  p.gpr = gpr;
+  p.n = n;
+  p.d = d;
+  p.gs = d / gpr;
+  p.T = T;
+  p.task = task;
+  p.ntask = ntask;
+  p.check = check;
+  return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sk_abi_version(void) { return SK_ABI_VERSION; }
+
+const char* sk_status_string(sk_status s) {
+  switch (s) {
+    case SK_OK: return "SK_OK";
+    case SK_ERR_INVALID_ARG: return "SK_ERR_INVALID_ARG";
+    case SK_ERR_UNSUPPORTED: return "SK_ERR_UNSUPPORTED";
+    case SK_ERR_CUDA: return "SK_ERR_CUDA";
+    case SK_ERR_DEVICE_CHECK: return "SK_ERR_DEVICE_CHECK";
+  }
+  return "SK_ERR_UNKNOWN";
+}
+
+const char* sk_last_error(void) { return g_last_error.c_str(); }
+
+size_t sk_packed_row_bytes(int64_t d, int bits) {
+  if (d % 32 != 0) return 0;
+  return row_bytes(d, bits);
+}
+
+size_t sk_packed_bytes(int64_t n, int64_t d, int bits) {
+  if (n < 0) return 0;
+  return (size_t)n * sk_packed_row_bytes(d, bits);
+}
+
+sk_status sk_pack(const uint8_t* idx, int64_t n, int64_t d, int bits, void* packed, size_t packed_bytes,
+                  sk_stream_t stream) {
+  g_last_error.clear();
+  if (bits < 2 || bits > 4) return fail(SK_ERR_INVALID_ARG, "bits must be 2, 3 or 4 (got %d)", bits);
+  if (n < 0 || d < 32 || d % 32 != 0 || n >= kMaxDim || d >= kMaxDim)
+    return fail(SK_ERR_INVALID_ARG, "need n >= 0 and d a positive multiple of 32 (n=%lld, d=%lld)", (long long)n, (long long)d);
+  const size_t need = sk_packed_bytes(n, d, bits);
+  if (packed_bytes < need) return fail(SK_ERR_INVALID_ARG, "packed buffer holds %zu bytes, need %zu", packed_bytes, need);
+  if (n == 0) return ok();
+  if (!idx || !packed) return fail(SK_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(idx) || !aligned16(packed)) return fail(SK_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (overlaps(idx, (size_t)(n * d), packed, need)) return fail(SK_ERR_INVALID_ARG, "idx and packed overlap");
+  unsigned int* check = nullptr;
+  sk_status st = device_state(&check);
+  if (st != SK_OK) return st;
+  cudaError_t e = sk::launch_pack(idx, n, d, bits, static_cast<uint8_t*>(packed), (int64_t)row_bytes(d, bits), check,
+                                  reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ok() : cuda_fail(e, "pack kernel launch");
+}
+
+sk_status sk_unpack(const void* packed, int64_t n, int64_t d, int bits, uint8_t* idx, sk_stream_t stream) {
+  g_last_error.clear();
+  if (bits < 2 || bits > 4) return fail(SK_ERR_INVALID_ARG, "bits must be 2, 3 or 4 (got %d)", bits);
+  if (n < 0 || d < 32 || d % 32 != 0 || n >= kMaxDim || d >= kMaxDim)
+    return fail(SK_ERR_INVALID_ARG, "need n >= 0 and d a positive multiple of 32 (n=%lld, d=%lld)", (long long)n, (long long)d);
+  if (n == 0) return ok();
+  if (!idx || !packed) return fail(SK_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(idx) || !aligned16(packed)) return fail(SK_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (overlaps(idx, (size_t)(n * d), packed, sk_packed_bytes(n, d, bits))) return fail(SK_ERR_INVALID_ARG, "idx and packed overlap");
+  unsigned int* check = nullptr;
+  sk_status st = device_state(&check);
+  if (st != SK_OK) return st;
+  cudaError_t e = sk::launch_unpack(static_cast<const uint8_t*>(packed), n, d, bits, (int64_t)row_bytes(d, bits), idx,
+                                    reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ok() : cuda_fail(e, "unpack kernel launch");
+}
+
+sk_status sk_dequant(const void* packed, const uint16_t* lut, int bits, int gpr, int64_t n, int64_t d, int task,
+                     int ntask, uint16_t* theta, sk_stream_t stream) {
+  g_last_error.clear();
+  sk_status st = check_shape(bits, gpr, n, d, 0, ntask);
+  if (st != SK_OK) return st;
+  if (task < 0 || task >= ntask) return fail(SK_ERR_INVALID_ARG, "task %d outside [0, %d)", task, ntask);
+  if (!packed || !lut || !theta) return fail(SK_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(packed) || !aligned16(lut) || !aligned16(theta)) return fail(SK_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  const size_t lut_bytes = (size_t)ntask * n * gpr * (1u << bits) * 2;
+  if (overlaps(theta, (size_t)(n * d * 2), packed, sk_packed_bytes(n, d, bits)) || overlaps(theta, (size_t)(n * d * 2), lut, lut_bytes))
+    return fail(SK_ERR_INVALID_ARG, "theta overlaps an input");
+  unsigned int* check = nullptr;
+  st = device_state(&check);
+  if (st != SK_OK) return st;
+  sk::Problem p = make_problem(packed, lut, bits, gpr, n, d, 0, nullptr, ntask, check);
+  cudaError_t e = sk::launch_dequant(p, task, theta, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ok() : cuda_fail(e, "dequant kernel launch");
+}
+
+size_t sk_workspace_bytes(int op, int64_t n, int64_t d, int bits, int gpr, int64_t T, int ntask) {
+  (void)n; (void)d; (void)bits; (void)gpr; (void)T; (void)ntask;
+  if (op < SK_OP_FWD || op > SK_OP_BWD_LUT) return 0;
+  return 0;
+}
+
+static sk_status check_layer_buffers(const void* packed, const uint16_t* lut, bool need_lut, int bits, int gpr,
+                                     int64_t n, int64_t d, int64_t T, const int32_t* task, int ntask,
+                                     const void* in, size_t in_bytes, const void* in2, size_t in2_bytes,
+                                     const void* out, size_t out_bytes) {
+  if (!packed || (need_lut && !lut) || !in || !out || (in2_bytes && !in2))
+    return fail(SK_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(packed) || (need_lut && !aligned16(lut)) || !aligned16(in) || !aligned16(out) || (in2 && !aligned16(in2)))
+    return fail(SK_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  const size_t pk = sk_packed_bytes(n, d, bits);
+  const size_t lb = need_lut ? (size_t)ntask * n * gpr * (1u << bits) * 2 : 0;
+  const size_t tb = task ? (size_t)T * 4 : 0;
+  if (overlaps(out, out_bytes, packed, pk) || overlaps(out, out_bytes, lut, lb) || overlaps(out, out_bytes, in, in_bytes) ||
+      overlaps(out, out_bytes, in2, in2_bytes) || overlaps(out, out_bytes, task, tb))
+    return fail(SK_ERR_INVALID_ARG, "output overlaps an input");
+  return SK_OK;
+}
+
+sk_status sk_linear_fwd(const void* packed, const uint16_t* lut, int bits, int gpr, int64_t n, int64_t d,
+                        const uint16_t* X, int64_t T, const int32_t* task, int ntask, uint16_t* Y,
+                        void* workspace, size_t workspace_bytes, sk_stream_t stream) {
+  g_last_error.clear();
+  (void)workspace;
+  sk_status st = check_shape(bits, gpr, n, d, T, ntask);
+  if (st != SK_OK) return st;
+  if (T == 0) return ok();
+  st = check_layer_buffers(packed, lut, true, bits, gpr, n, d, T, task, ntask, X, (size_t)(T * d * 2), nullptr, 0, Y,
+                           (size_t)(T * n * 2));
+  if (st != SK_OK) return st;
+  if (workspace_bytes < sk_workspace_bytes(SK_OP_FWD, n, d, bits, gpr, T, ntask))
+    return fail(SK_ERR_INVALID_ARG, "workspace too small");
+  unsigned int* check = nullptr;
+  st = device_state(&check);
+  if (st != SK_OK) return st;
+  sk::Problem p = make_problem(packed, lut, bits, gpr, n, d, T, task, ntask, check);
+  cudaError_t e = sk::launch_gemv_fwd(p, X, Y, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ok() : cuda_fail(e, "forward kernel launch");
+}
+
+sk_status sk_linear_bwd_input(const void* packed, const uint16_t* lut, int bits, int gpr, int64_t n, int64_t d,
+                              const uint16_t* dY, int64_t T, const int32_t* task, int ntask, uint16_t* dX,
+                              void* workspace, size_t workspace_bytes, sk_stream_t stream) {
+  g_last_error.clear();
+  (void)workspace;
+  sk_status st = check_shape(bits, gpr, n, d, T, ntask);
+  if (st != SK_OK) return st;
+  if (T == 0) return ok();
+  st = check_layer_buffers(packed, lut, true, bits, gpr, n, d, T, task, ntask, dY, (size_t)(T * n * 2), nullptr, 0, dX,
+                           (size_t)(T * d * 2));
+  if (st != SK_OK) return st;
+  if (workspace_bytes < sk_workspace_bytes(SK_OP_BWD_INPUT, n, d, bits, gpr, T, ntask))
+    return fail(SK_ERR_INVALID_ARG, "workspace too small");
+  unsigned int* check = nullptr;
+  st = device_state(&check);
+  if (st != SK_OK) return st;
+  sk::Problem p = make_problem(packed, lut, bits, gpr, n, d, T, task, ntask, check);
+  cudaError_t e = sk::launch_simt_bwd_input(p, dY, dX, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ok() : cuda_fail(e, "input-gradient kernel launch");
+}
+
+sk_status sk_linear_bwd_lut(const void* packed, int bits, int gpr, int64_t n, int64_t d, const uint16_t* X,
+                            const uint16_t* dY, int64_t T, const int32_t* task, int ntask, float* dlut,
+                            int accumulate, void* workspace, size_t workspace_bytes, sk_stream_t stream) {
+  g_last_error.clear();
+  (void)workspace;
+  sk_status st = check_shape(bits, gpr, n, d, T, ntask);
+  if (st != SK_OK) return st;
+  if (accumulate != 0 && accumulate != 1) return fail(SK_ERR_INVALID_ARG, "accumulate must be 0 or 1");
+  const size_t dlut_bytes = (size_t)ntask * n * gpr * (1u << bits) * 4;
+  if (!dlut) return fail(SK_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(dlut)) return fail(SK_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (T == 0) {
+    if (accumulate) return ok();
+    cudaError_t e = cudaMemsetAsync(dlut, 0, dlut_bytes, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ok() : cuda_fail(e, "cudaMemsetAsync(dlut)");
+  }
+  st = check_layer_buffers(packed, nullptr, false, bits, gpr, n, d, T, task, ntask, X, (size_t)(T * d * 2), dY,
+                           (size_t)(T * n * 2), dlut, dlut_bytes);
+  if (st != SK_OK) return st;
+  if (workspace_bytes < sk_workspace_bytes(SK_OP_BWD_LUT, n, d, bits, gpr, T, ntask))
+    return fail(SK_ERR_INVALID_ARG, "workspace too small");
+  unsigned int* check = nullptr;
+  st = device_state(&check);
+  if (st != SK_OK) return st;
+  sk::Problem p = make_problem(packed, nullptr, bits, gpr, n, d, T, task, ntask, check);
+  cudaError_t e = sk::launch_simt_bwd_lut(p, X, dY, dlut, accumulate, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ok() : cuda_fail(e, "LUT-gradient kernel launch");
+}
+
+sk_status sk_device_check(uint32_t* flags, int clear, sk_stream_t stream) {
+  g_last_error.clear();
+  if (!flags) return fail(SK_ERR_INVALID_ARG, "null pointer");
+  unsigned int* check = nullptr;
+  sk_status st = device_state(&check);
+  if (st != SK_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned int host = 0;
+  cudaError_t e = cudaMemcpyAsync(&host, check, sizeof host, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess && clear) e = cudaMemsetAsync(check, 0, sizeof host, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device check word");
+  *flags = host;
+  if (host) return fail(SK_ERR_DEVICE_CHECK, "device check word 0x%x", host);
+  return SK_OK;
+}
+
+}  // extern "C"

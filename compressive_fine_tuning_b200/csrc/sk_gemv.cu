@@ -1,0 +1,129 @@
+// Decode forward on the CUDA cores: Y[t][i] = sum_j X[t][j] * Theta_hat[i][j]
+// for a handful of tokens ("SpaLLM: Unified Compressive Adaptation of LLMs
+// with Sketching", section 2.3: one compressed matmul per layer; section 3.2,
+// Table 5: decode is where the single-tower layer pays off).
+//
+// Work split: a warp owns R weight rows and splits their columns across its
+// lanes; each lane walks pairs of 32-column chunks (one 16/8/12-byte index
+// load per chunk, consecutive lanes on consecutive chunks so a warp-wide load
+// is one contiguous span of the row), dequantises them through register LUTs
+// and accumulates R x TT fp32 dot products with bf16 x fp32 fused multiply-adds.
+// A warp-shuffle tree then reduces the lane partial sums.  Tokens are taken TT
+// at a time; tokens with different LUT sets re-dequantise the chunk.
+#include "sk_internal.cuh"
+
+namespace sk {
+namespace {
+
+constexpr int kWarps = 4;
+
+template <int BITS, int R, int TT>
+__global__ void __launch_bounds__(kWarps * 32) gemv_fwd_kernel(Problem p, const uint16_t* __restrict__ X,
+                                                               uint16_t* __restrict__ Y) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row0 = ((int64_t)blockIdx.x * kWarps + warp) * R;
+  if (row0 >= p.n) return;
+  const int64_t chunks = p.d / 32;
+  const int64_t cpg = p.gs / 32;
+  const uint8_t* rows[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) rows[r] = p.packed + (row0 + r < p.n ? row0 + r : p.n - 1) * p.row_bytes;
+
+  for (int64_t t0 = 0; t0 < p.T; t0 += TT) {
+    const int nt = (int)(p.T - t0 < TT ? p.T - t0 : TT);
+    int taus[TT];
+#pragma unroll
+    for (int u = 0; u < TT; ++u) taus[u] = (u < nt) ? token_task(p.task, t0 + u, p.ntask, p.check) : -1;
+
+    float acc[R][TT];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int u = 0; u < TT; ++u) acc[r][u] = 0.f;
+
+    for (int64_t c = lane; c < chunks; c += 32) {
+      const int64_t g = c / cpg;
+      Chunk<BITS> ch[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) ch[r] = load_chunk<BITS>(rows[r], c);
+      uint32_t w[R][16];
+      int cur = -2;
+#pragma unroll
+      for (int u = 0; u < TT; ++u) {
+        if (taus[u] < 0) continue;
+        if (taus[u] != cur) {
+          cur = taus[u];
+#pragma unroll
+          for (int r = 0; r < R; ++r) {
+            LutRegs<BITS> L;
+            load_lut<BITS>(lut_ptr(p, cur, (row0 + r < p.n ? row0 + r : p.n - 1), g), L);
+            dequant_chunk<BITS>(ch[r], L, w[r]);
+          }
+        }
+        const uint4* xp = reinterpret_cast<const uint4*>(X + (t0 + u) * p.d + c * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 xv = __ldg(xp + q);
+#pragma unroll
+          for (int r = 0; r < R; ++r) {
+            float a = acc[r][u];
+            a = fma_bf16x2(w[r][4 * q + 0], xv.x, a);
+            a = fma_bf16x2(w[r][4 * q + 1], xv.y, a);
+            a = fma_bf16x2(w[r][4 * q + 2], xv.z, a);
+            a = fma_bf16x2(w[r][4 * q + 3], xv.w, a);
+            acc[r][u] = a;
+          }
+        }
+      }
+    }
+
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+#pragma unroll
+      for (int u = 0; u < TT; ++u) {
+        float v = acc[r][u];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        acc[r][u] = v;
+      }
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        if (row0 + r >= p.n) continue;
+#pragma unroll
+        for (int u = 0; u < TT; ++u) {
+          if (u >= nt) continue;
+          __nv_bfloat16 b = __float2bfloat16_rn(acc[r][u]);
+          Y[(t0 + u) * p.n + row0 + r] = *reinterpret_cast<uint16_t*>(&b);
+        }
+      }
+    }
+  }
+}
+
+template <int BITS, int R, int TT>
+cudaError_t launch(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStream_t s) {
+  const int64_t rows_per_cta = (int64_t)kWarps * R;
+  const unsigned grid = (unsigned)((p.n + rows_per_cta - 1) / rows_per_cta);
+  gemv_fwd_kernel<BITS, R, TT><<<grid, kWarps * 32, 0, s>>>(p, X, Y);
+  return cudaGetLastError();
+}
+
+template <int BITS>
+cudaError_t launch_bits(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStream_t s) {
+  if (p.T == 1) return launch<BITS, 2, 1>(p, X, Y, s);
+  return launch<BITS, 2, 4>(p, X, Y, s);
+}
+
+}  // namespace
+
+cudaError_t launch_gemv_fwd(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStream_t s) {
+  switch (p.bits) {
+    case 2: return launch_bits<2>(p, X, Y, s);
+    case 3: return launch_bits<3>(p, X, Y, s);
+    default: return launch_bits<4>(p, X, Y, s);
+  }
+}
+
+}  // namespace sk

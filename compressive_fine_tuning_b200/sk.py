@@ -1,0 +1,252 @@
+"""Thin Python binding of libsk.so (the sketched linear layer's C ABI).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  PyTorch supplies device memory and the current stream.  Importing
+this module fails loudly when the library has not been built; there is no
+fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsk.so")
+
+SK_OK = 0
+SK_OP_FWD, SK_OP_BWD_INPUT, SK_OP_BWD_LUT = 0, 1, 2
+SK_CHECK_TASK_RANGE = 1
+SK_CHECK_INDEX_RANGE = 2
+
+EXPORTED = (
+    "sk_abi_version", "sk_status_string", "sk_last_error", "sk_packed_row_bytes", "sk_packed_bytes",
+    "sk_pack", "sk_unpack", "sk_dequant", "sk_workspace_bytes", "sk_linear_fwd", "sk_linear_bwd_input",
+    "sk_linear_bwd_lut", "sk_device_check",
+)
+
+
+class SketchError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(message)
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"{_LIB_PATH} is missing: build it with `python -m compressive_fine_tuning_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    sigs = {
+        "sk_abi_version": ([], i32),
+        "sk_status_string": ([i32], ctypes.c_char_p),
+        "sk_last_error": ([], ctypes.c_char_p),
+        "sk_packed_row_bytes": ([i64, i32], sz),
+        "sk_packed_bytes": ([i64, i64, i32], sz),
+        "sk_pack": ([vp, i64, i64, i32, vp, sz, vp], i32),
+        "sk_unpack": ([vp, i64, i64, i32, vp, vp], i32),
+        "sk_dequant": ([vp, vp, i32, i32, i64, i64, i32, i32, vp, vp], i32),
+        "sk_workspace_bytes": ([i32, i64, i64, i32, i32, i64, i32], sz),
+        "sk_linear_fwd": ([vp, vp, i32, i32, i64, i64, vp, i64, vp, i32, vp, vp, sz, vp], i32),
+        "sk_linear_bwd_input": ([vp, vp, i32, i32, i64, i64, vp, i64, vp, i32, vp, vp, sz, vp], i32),
+        "sk_linear_bwd_lut": ([vp, i32, i32, i64, i64, vp, vp, i64, vp, i32, vp, i32, vp, sz, vp], i32),
+        "sk_device_check": ([ctypes.POINTER(ctypes.c_uint32), i32, vp], i32),
+    }
+    for name, (args, res) in sigs.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+lib = _load()
+
+
+def _check(status: int) -> None:
+    if status != SK_OK:
+        name = lib.sk_status_string(status).decode()
+        raise SketchError(status, f"{name}: {lib.sk_last_error().decode()}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t: torch.Tensor, dtype: torch.dtype, name: str, ndim: Optional[int] = None) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions")
+
+
+def packed_row_bytes(d: int, bits: int) -> int:
+    return int(lib.sk_packed_row_bytes(d, bits))
+
+
+def packed_bytes(n: int, d: int, bits: int) -> int:
+    return int(lib.sk_packed_bytes(n, d, bits))
+
+
+def workspace_bytes(op: int, n: int, d: int, bits: int, gpr: int, T: int, ntask: int) -> int:
+    return int(lib.sk_workspace_bytes(op, n, d, bits, gpr, T, ntask))
+
+
+def _workspace(op, n, d, bits, gpr, T, ntask, device):
+    nb = workspace_bytes(op, n, d, bits, gpr, T, ntask)
+    if nb == 0:
+        return None, 0
+    return torch.empty(nb, dtype=torch.uint8, device=device), nb
+
+
+def pack(idx: torch.Tensor, bits: int, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """uint8 [n, d] indices -> uint8 [n, packed_row_bytes] packed rows (on the GPU)."""
+    _need(idx, torch.uint8, "idx", 2)
+    n, d = idx.shape
+    rb = packed_row_bytes(d, bits)
+    if out is None:
+        out = torch.empty((n, max(rb, 1)), dtype=torch.uint8, device=idx.device)
+    _need(out, torch.uint8, "out")
+    _check(lib.sk_pack(_ptr(idx), n, d, bits, _ptr(out), out.numel(), _stream(idx.device)))
+    return out
+
+
+def unpack(packed: torch.Tensor, n: int, d: int, bits: int) -> torch.Tensor:
+    _need(packed, torch.uint8, "packed")
+    out = torch.empty((n, d), dtype=torch.uint8, device=packed.device)
+    _check(lib.sk_unpack(_ptr(packed), n, d, bits, _ptr(out), _stream(packed.device)))
+    return out
+
+
+def _lut_shape(lut: torch.Tensor, bits: int):
+    _need(lut, torch.float16, "lut", 4)
+    ntask, n, gpr, k = lut.shape
+    if k != (1 << bits):
+        raise ValueError(f"lut's last dimension must be 2**bits = {1 << bits}")
+    return ntask, n, gpr
+
+
+def dequant(packed: torch.Tensor, lut: torch.Tensor, bits: int, d: int, task: int = 0) -> torch.Tensor:
+    """Dense bf16 [n, d] effective weight of LUT set `task` (test / comparison aid)."""
+    ntask, n, gpr = _lut_shape(lut, bits)
+    _need(packed, torch.uint8, "packed")
+    out = torch.empty((n, d), dtype=torch.bfloat16, device=lut.device)
+    _check(lib.sk_dequant(_ptr(packed), _ptr(lut), bits, gpr, n, d, task, ntask, _ptr(out), _stream(lut.device)))
+    return out
+
+
+def _task_arg(task: Optional[torch.Tensor], T: int):
+    if task is None:
+        return None
+    _need(task, torch.int32, "task", 1)
+    if task.numel() != T:
+        raise ValueError("task must hold one id per token")
+    return task
+
+
+def linear_fwd(packed: torch.Tensor, lut: torch.Tensor, bits: int, X: torch.Tensor,
+               task: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Y [T, n] = X Theta_hat^T (bf16 in, bf16 out, fp32 accumulation)."""
+    ntask, n, gpr = _lut_shape(lut, bits)
+    _need(X, torch.bfloat16, "X", 2)
+    _need(packed, torch.uint8, "packed")
+    T, d = X.shape
+    task = _task_arg(task, T)
+    if out is None:
+        out = torch.empty((T, n), dtype=torch.bfloat16, device=X.device)
+    _need(out, torch.bfloat16, "out", 2)
+    ws, nb = _workspace(SK_OP_FWD, n, d, bits, gpr, T, ntask, X.device)
+    _check(lib.sk_linear_fwd(_ptr(packed), _ptr(lut), bits, gpr, n, d, _ptr(X), T, _ptr(task), ntask,
+                             _ptr(out), _ptr(ws), nb, _stream(X.device)))
+    return out
+
+
+def linear_bwd_input(packed: torch.Tensor, lut: torch.Tensor, bits: int, d: int, dY: torch.Tensor,
+                     task: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """dX [T, d] = dY Theta_hat."""
+    ntask, n, gpr = _lut_shape(lut, bits)
+    _need(dY, torch.bfloat16, "dY", 2)
+    _need(packed, torch.uint8, "packed")
+    T = dY.shape[0]
+    if dY.shape[1] != n:
+        raise ValueError("dY must be [T, n]")
+    task = _task_arg(task, T)
+    if out is None:
+        out = torch.empty((T, d), dtype=torch.bfloat16, device=dY.device)
+    _need(out, torch.bfloat16, "out", 2)
+    ws, nb = _workspace(SK_OP_BWD_INPUT, n, d, bits, gpr, T, ntask, dY.device)
+    _check(lib.sk_linear_bwd_input(_ptr(packed), _ptr(lut), bits, gpr, n, d, _ptr(dY), T, _ptr(task), ntask,
+                                   _ptr(out), _ptr(ws), nb, _stream(dY.device)))
+    return out
+
+
+def linear_bwd_lut(packed: torch.Tensor, bits: int, gpr: int, X: torch.Tensor, dY: torch.Tensor,
+                   task: Optional[torch.Tensor] = None, ntask: int = 1, out: Optional[torch.Tensor] = None,
+                   accumulate: bool = False) -> torch.Tensor:
+    """dlut [ntask, n, gpr, k] fp32: the binned dY^T X of the corrected Eq. 6."""
+    _need(X, torch.bfloat16, "X", 2)
+    _need(dY, torch.bfloat16, "dY", 2)
+    _need(packed, torch.uint8, "packed")
+    T, d = X.shape
+    n = dY.shape[1]
+    if dY.shape[0] != T:
+        raise ValueError("X and dY must have the same number of tokens")
+    task = _task_arg(task, T)
+    k = 1 << bits
+    if out is None:
+        out = torch.empty((ntask, n, gpr, k), dtype=torch.float32, device=X.device)
+    _need(out, torch.float32, "out")
+    ws, nb = _workspace(SK_OP_BWD_LUT, n, d, bits, gpr, T, ntask, X.device)
+    _check(lib.sk_linear_bwd_lut(_ptr(packed), bits, gpr, n, d, _ptr(X), _ptr(dY), T, _ptr(task), ntask,
+                                 _ptr(out), int(accumulate), _ptr(ws), nb, _stream(X.device)))
+    return out
+
+
+def device_check(clear: bool = True, device=None) -> int:
+    """Synchronise and return the device check word (SK_CHECK_* bits)."""
+    device = torch.device("cuda") if device is None else torch.device(device)
+    flags = ctypes.c_uint32(0)
+    st = lib.sk_device_check(ctypes.byref(flags), int(clear), _stream(device))
+    if st not in (SK_OK, 4):
+        _check(st)
+    return int(flags.value)
+
+
+class SketchedLinearFunction(torch.autograd.Function):
+    """Y = X Theta_hat^T with gradients for X and for the LUT values only."""
+
+    @staticmethod
+    def forward(ctx, X, lut, packed, bits, task):
+        Y = linear_fwd(packed, lut, bits, X.contiguous(), task)
+        ctx.save_for_backward(X, lut, packed, task if task is not None else torch.empty(0))
+        ctx.bits = bits
+        ctx.has_task = task is not None
+        return Y
+
+    @staticmethod
+    def backward(ctx, dY):
+        X, lut, packed, task = ctx.saved_tensors
+        task = task if ctx.has_task else None
+        dY = dY.contiguous().to(torch.bfloat16)
+        dX = dlut = None
+        if ctx.needs_input_grad[0]:
+            dX = linear_bwd_input(packed, lut, ctx.bits, X.shape[1], dY, task)
+        if ctx.needs_input_grad[1]:
+            ntask, n, gpr, _ = lut.shape
+            dlut = linear_bwd_lut(packed, ctx.bits, gpr, X, dY, task, ntask).to(lut.dtype)
+        return dX, dlut, None, None, None
+
+
+def sketched_linear(X: torch.Tensor, lut: torch.Tensor, packed: torch.Tensor, bits: int,
+                    task: Optional[torch.Tensor] = None) -> torch.Tensor:
+    return SketchedLinearFunction.apply(X, lut, packed, bits, task)

@@ -1,0 +1,178 @@
+/*
+ * sk.h -- C ABI of the sketched linear layer (libsk.so, B200 / sm_100a).
+ *
+ * The layer ("SpaLLM: Unified Compressive Adaptation of LLMs with Sketching",
+ * section 2.2, Eq. 1): each row of an n x d weight is split into `gpr`
+ * contiguous groups of gs = d / gpr columns ("groups per row"); every group
+ * keeps a lookup table (LUT) of k = 2^bits fp16 values and a frozen one-hot
+ * sketching matrix, stored as an index map idx[i][j] in [0, k).  The
+ * effective weight is
+ *
+ *     Theta_hat[i][j] = lut[task][i][j / gs][idx[i][j]].
+ *
+ * Several LUT sets ("tasks") may share one index map (section 2.3); token t
+ * then uses lut[task[t]].
+ *
+ * Data layouts (all row-major and contiguous, device memory unless stated):
+ *   packed : the index map in the packed format below, sk_packed_bytes() bytes.
+ *   lut    : IEEE fp16 bits, [ntask][n][gpr][k].
+ *   X      : bf16 bits, [T][d]        (layer input, one row per token).
+ *   Y, dY  : bf16 bits, [T][n]        (layer output and its gradient).
+ *   dX     : bf16 bits, [T][d].
+ *   dlut   : fp32, [ntask][n][gpr][k] (gradient of the loss w.r.t. lut).
+ *   task   : int32 [T] task id per token, or NULL (every token uses LUT set 0).
+ *
+ * Packed index format (this library's own; the pages leave index storage
+ * open): each row is packed on its own and zero-padded to a multiple of 16
+ * bytes (sk_packed_row_bytes).  4-bit: two per byte, index j in nibble (j & 1)
+ * of byte j >> 1, low nibble first.  2-bit: four per byte, index j at bits
+ * 2*(j & 3) of byte j >> 2.  3-bit: 32 indices per three little-endian uint32
+ * words; index j of a 32-index chunk starts at bit 3*(j mod 32) of the 96-bit
+ * chunk.
+ *
+ * Shape rules, checked on the host before anything is launched:
+ *   bits in {2, 3, 4}; n >= 1 and n % 8 == 0; d >= 32; gpr >= 1;
+ *   d % gpr == 0 and (d / gpr) % 32 == 0 (so every 32-column chunk lies in one
+ *   group); T >= 0 (T == 0 launches nothing and returns SK_OK); ntask >= 1.
+ *
+ * Ownership: the caller allocates and owns every buffer, including any
+ * workspace (size from sk_workspace_bytes).  Device pointers must be 16-byte
+ * aligned.  Outputs must not overlap inputs.  The library keeps no state
+ * besides a device-side check word (sk_device_check) and never allocates
+ * device memory.
+ *
+ * Errors: a non-OK status means nothing was launched, except SK_ERR_CUDA,
+ * which reports a failed launch (the CUDA error string is in sk_last_error()).
+ * Errors of kernels that already ran asynchronously surface at the caller's
+ * next synchronisation, as usual in CUDA.  Data checks that need the device
+ * (a task id outside [0, ntask), an index >= 2^bits given to sk_pack) do not
+ * stop the kernel: the affected output is written as zero / masked and a bit
+ * is set in the device check word, which sk_device_check() reads.
+ *
+ * Streams: every call is asynchronous on the given stream (NULL = the legacy
+ * default stream).
+ */
+#ifndef SK_H_
+#define SK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SK_ABI_VERSION 1
+
+typedef struct CUstream_st* sk_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  SK_OK = 0,
+  SK_ERR_INVALID_ARG = 1,  /* bad pointer, size, shape or overlap          */
+  SK_ERR_UNSUPPORTED = 2,  /* valid but not handled (e.g. no sm_100 device) */
+  SK_ERR_CUDA = 3,         /* a CUDA call or launch failed                   */
+  SK_ERR_DEVICE_CHECK = 4  /* sk_device_check found a flagged input          */
+} sk_status;
+
+/* Device check word bits (sk_device_check). */
+#define SK_CHECK_TASK_RANGE 1u   /* a task id outside [0, ntask) was seen      */
+#define SK_CHECK_INDEX_RANGE 2u  /* sk_pack saw an index >= 2^bits             */
+
+/* Operation selectors for sk_workspace_bytes. */
+#define SK_OP_FWD 0
+#define SK_OP_BWD_INPUT 1
+#define SK_OP_BWD_LUT 2
+
+int sk_abi_version(void);
+const char* sk_status_string(sk_status s);
+/* Detail of the last non-OK status returned on this host thread ("" if none). */
+const char* sk_last_error(void);
+
+/* Bytes of one packed row: ceil(d * bits / 8) rounded up to 16.  0 if bits or d is invalid. */
+size_t sk_packed_row_bytes(int64_t d, int bits);
+/* n * sk_packed_row_bytes(d, bits).  0 if the arguments are invalid. */
+size_t sk_packed_bytes(int64_t n, int64_t d, int bits);
+
+/*
+ * sk_pack: idx (device uint8 [n][d], values < 2^bits) -> packed (device,
+ * packed_bytes >= sk_packed_bytes(n, d, bits)).  Padding bytes are written as
+ * zero.  An index >= 2^bits is masked to its low bits and sets
+ * SK_CHECK_INDEX_RANGE.  This is step a0 (off the timed path): it encodes the
+ * one-hot sketching matrix of Eq. 1 as its column indices.
+ */
+sk_status sk_pack(const uint8_t* idx, int64_t n, int64_t d, int bits,
+                  void* packed, size_t packed_bytes, sk_stream_t stream);
+
+/* sk_unpack: the inverse of sk_pack (device packed -> device uint8 [n][d]). */
+sk_status sk_unpack(const void* packed, int64_t n, int64_t d, int bits,
+                    uint8_t* idx, sk_stream_t stream);
+
+/*
+ * sk_dequant: writes the dense effective weight of LUT set `task` as bf16 bits
+ * [n][d] (Eq. 1 with groups per row), each value the round-to-nearest-even
+ * bf16 of the fp16 table entry.  The fused kernels use exactly these values.
+ * Meant for tests and for a dense-GEMM comparison; not on the hot path.
+ */
+sk_status sk_dequant(const void* packed, const uint16_t* lut, int bits, int gpr,
+                     int64_t n, int64_t d, int task, int ntask,
+                     uint16_t* theta, sk_stream_t stream);
+
+/*
+ * Workspace bytes that the call selected by `op` (SK_OP_*) needs for these
+ * shapes; 0 means no workspace (a NULL workspace is then fine).
+ */
+size_t sk_workspace_bytes(int op, int64_t n, int64_t d, int bits, int gpr,
+                          int64_t T, int ntask);
+
+/*
+ * sk_linear_fwd: Y = X Theta_hat^T, token t with LUT set task[t].
+ * SpaLLM section 2.3: one compressed matmul per layer, no adapter branch.
+ * Accumulation is fp32; weights enter the tensor cores as bf16 (the RNE
+ * rounding of the fp16 table values, as sk_dequant writes them); Y is rounded
+ * to bf16 (RNE).
+ */
+sk_status sk_linear_fwd(const void* packed, const uint16_t* lut, int bits, int gpr,
+                        int64_t n, int64_t d, const uint16_t* X, int64_t T,
+                        const int32_t* task, int ntask, uint16_t* Y,
+                        void* workspace, size_t workspace_bytes, sk_stream_t stream);
+
+/*
+ * sk_linear_bwd_input: dX = dY Theta_hat (chain rule through the frozen
+ * sketch; the layer has to pass gradients back to earlier layers).  Same
+ * precision rules as sk_linear_fwd.
+ */
+sk_status sk_linear_bwd_input(const void* packed, const uint16_t* lut, int bits, int gpr,
+                              int64_t n, int64_t d, const uint16_t* dY, int64_t T,
+                              const int32_t* task, int ntask, uint16_t* dX,
+                              void* workspace, size_t workspace_bytes, sk_stream_t stream);
+
+/*
+ * sk_linear_bwd_lut: the LUT gradient of the corrected Eq. 6 ("Sketch to
+ * Adapt" OpenReview discussion, reply Q1): dL/dw = dL/dy (M X)^T, i.e.
+ *
+ *     dlut[task][i][g][c] = sum over tokens t with task[t] == task and
+ *                           columns j of group g with idx[i][j] == c
+ *                           of dY[t][i] * X[t][j].
+ *
+ * The loss is linear in the LUT, so no LUT values are needed.  The dense
+ * n x d gradient is never written to memory.  accumulate = 0 overwrites dlut,
+ * 1 adds to it.  fp32 throughout; the result is deterministic (no float
+ * atomics).
+ */
+sk_status sk_linear_bwd_lut(const void* packed, int bits, int gpr, int64_t n, int64_t d,
+                            const uint16_t* X, const uint16_t* dY, int64_t T,
+                            const int32_t* task, int ntask, float* dlut, int accumulate,
+                            void* workspace, size_t workspace_bytes, sk_stream_t stream);
+
+/*
+ * sk_device_check: synchronises `stream`, stores the device check word
+ * (SK_CHECK_* bits, 0 = nothing flagged) in *flags and clears it if `clear`.
+ * Returns SK_ERR_DEVICE_CHECK when any bit was set, else SK_OK.
+ */
+sk_status sk_device_check(uint32_t* flags, int clear, sk_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SK_H_ */

@@ -1,0 +1,132 @@
+"""The C-ABI library loads, exports every declared symbol, and validates
+arguments on the host before touching a device (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from compressive_fine_tuning_b200 import sk
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sk.h")
+
+SK_OK, SK_ERR_INVALID_ARG, SK_ERR_UNSUPPORTED, SK_ERR_CUDA = 0, 1, 2, 3
+
+# fake, 16-byte aligned, non-overlapping "device" addresses: validation must
+# reject bad calls before any of them is dereferenced
+A = ctypes.c_void_p(0x10000000)
+B = ctypes.c_void_p(0x20000000)
+C = ctypes.c_void_p(0x30000000)
+D = ctypes.c_void_p(0x40000000)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sk_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_expected_calls():
+    names = declared_functions()
+    for must in ("sk_pack", "sk_linear_fwd", "sk_linear_bwd_input", "sk_linear_bwd_lut"):
+        assert must in names
+    assert set(names) == set(sk.EXPORTED)
+
+
+def test_every_declared_symbol_is_exported():
+    lib = ctypes.CDLL(sk._LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_abi_version_and_strings():
+    assert sk.lib.sk_abi_version() == 1
+    for code, name in [(0, b"SK_OK"), (1, b"SK_ERR_INVALID_ARG"), (2, b"SK_ERR_UNSUPPORTED"),
+                       (3, b"SK_ERR_CUDA"), (4, b"SK_ERR_DEVICE_CHECK"), (99, b"SK_ERR_UNKNOWN")]:
+        assert sk.lib.sk_status_string(code) == name
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("d", [32, 96, 160, 512, 1376, 4096, 5120, 11008, 13824, 28672])
+def test_packed_sizes_match_oracle(bits, d):
+    assert sk.packed_row_bytes(d, bits) == oracle.row_stride_bytes(d, bits)
+    assert sk.packed_bytes(7, d, bits) == oracle.packed_bytes(7, d, bits)
+
+
+def test_packed_sizes_reject_bad_args():
+    assert sk.packed_row_bytes(33, 4) == 0
+    assert sk.packed_row_bytes(64, 5) == 0
+    assert sk.packed_bytes(-1, 64, 4) == 0
+
+
+def fwd(packed=A, lut=B, bits=4, gpr=1, n=256, d=512, X=C, T=4, task=None, ntask=1, Y=D, ws=None, wsb=0):
+    return sk.lib.sk_linear_fwd(packed, lut, bits, gpr, n, d, X, T, task, ntask, Y, ws, wsb, None)
+
+
+def bwd_in(packed=A, lut=B, bits=4, gpr=1, n=256, d=512, dY=C, T=4, task=None, ntask=1, dX=D):
+    return sk.lib.sk_linear_bwd_input(packed, lut, bits, gpr, n, d, dY, T, task, ntask, dX, None, 0, None)
+
+
+def bwd_lut(packed=A, bits=4, gpr=1, n=256, d=512, X=B, dY=C, T=4, task=None, ntask=1, dlut=D, acc=0):
+    return sk.lib.sk_linear_bwd_lut(packed, bits, gpr, n, d, X, dY, T, task, ntask, dlut, acc, None, 0, None)
+
+
+@pytest.mark.parametrize("call", [fwd, bwd_in, bwd_lut])
+@pytest.mark.parametrize("kw", [
+    dict(bits=1), dict(bits=5), dict(n=0), dict(n=12), dict(d=48), dict(d=0), dict(gpr=0), dict(gpr=3),
+    dict(gpr=32),  # 512 / 32 = 16 columns per group: not a multiple of 32
+    dict(T=-1), dict(ntask=0),
+])
+def test_bad_shapes_rejected(call, kw):
+    assert call(**kw) == SK_ERR_INVALID_ARG
+    assert sk.lib.sk_last_error() != b""
+
+
+def test_bad_pointers_rejected():
+    assert fwd(packed=None) == SK_ERR_INVALID_ARG
+    assert fwd(lut=None) == SK_ERR_INVALID_ARG
+    assert fwd(X=None) == SK_ERR_INVALID_ARG
+    assert fwd(Y=None) == SK_ERR_INVALID_ARG
+    assert fwd(X=ctypes.c_void_p(0x30000008)) == SK_ERR_INVALID_ARG   # misaligned
+    assert bwd_in(dX=ctypes.c_void_p(0x40000004)) == SK_ERR_INVALID_ARG
+    assert bwd_lut(dlut=None) == SK_ERR_INVALID_ARG
+    assert bwd_lut(dY=None) == SK_ERR_INVALID_ARG
+    assert bwd_lut(acc=2) == SK_ERR_INVALID_ARG
+
+
+def test_overlapping_output_rejected():
+    # Y starts inside X's [T][d] bf16 range
+    assert fwd(X=C, Y=ctypes.c_void_p(0x30000000 + 1024)) == SK_ERR_INVALID_ARG
+    assert bwd_in(dY=C, dX=C) == SK_ERR_INVALID_ARG
+    assert bwd_lut(X=B, dlut=ctypes.c_void_p(0x20000000 + 16)) == SK_ERR_INVALID_ARG
+
+
+def test_empty_batch_is_a_no_op():
+    # T == 0 launches nothing, so it succeeds even without a device
+    assert fwd(T=0) == SK_OK
+    assert bwd_in(T=0) == SK_OK
+    assert bwd_lut(T=0, acc=1) == SK_OK
+
+
+def test_pack_validation():
+    L = sk.lib
+    assert L.sk_pack(A, 4, 64, 5, B, 4096, None) == SK_ERR_INVALID_ARG
+    assert L.sk_pack(A, 4, 48, 4, B, 4096, None) == SK_ERR_INVALID_ARG
+    assert L.sk_pack(A, 4, 64, 4, B, 16, None) == SK_ERR_INVALID_ARG           # buffer too small
+    assert L.sk_pack(A, 0, 64, 4, B, 0, None) == SK_OK                          # nothing to do
+    assert L.sk_pack(A, 4, 64, 4, ctypes.c_void_p(0x10000000 + 64), 4096, None) == SK_ERR_INVALID_ARG  # overlap
+    assert L.sk_unpack(A, 4, 64, 7, B, None) == SK_ERR_INVALID_ARG
+    assert L.sk_dequant(A, B, 4, 1, 256, 512, 1, 1, C, None) == SK_ERR_INVALID_ARG  # task outside [0, ntask)
+
+
+def test_valid_call_without_device_fails_loudly():
+    # the product path has no CPU fallback: with no usable device a valid call
+    # reports a CUDA / unsupported-device error instead of computing anything
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present")
+    assert fwd() in (SK_ERR_CUDA, SK_ERR_UNSUPPORTED)
+    assert bwd_in() in (SK_ERR_CUDA, SK_ERR_UNSUPPORTED)
+    assert bwd_lut() in (SK_ERR_CUDA, SK_ERR_UNSUPPORTED)
