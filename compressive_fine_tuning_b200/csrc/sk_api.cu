@@ -8,6 +8,7 @@
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <string>
 
@@ -80,6 +81,28 @@ size_t row_bytes(int64_t d, int bits) {
 }
 
 constexpr int64_t kMaxDim = int64_t(1) << 31;
+
+// Kernel choice for the forward.  SK_FWD_PATH=gemv|tc forces one path (for
+// measurements and tests); by default the tensor-core kernel takes every
+// single-LUT-set batch of at least kFwdTcMinT tokens on layers at least 128
+// columns wide.
+constexpr int64_t kFwdTcMinT = 2;
+
+int env_path(const char* name) {
+  const char* v = getenv(name);
+  if (v == nullptr) return 0;
+  if (strcmp(v, "gemv") == 0 || strcmp(v, "simt") == 0) return 1;
+  if (strcmp(v, "tc") == 0) return 2;
+  return 0;
+}
+
+bool use_tensor_cores_fwd(const sk::Problem& p) {
+  const bool tc_ok = (p.task == nullptr || p.ntask == 1) && p.d >= 128;
+  const int forced = env_path("SK_FWD_PATH");
+  if (forced == 1) return false;
+  if (forced == 2) return tc_ok;
+  return tc_ok && p.T >= kFwdTcMinT;
+}
 
 // Shape rules shared by the layer calls.
 sk_status check_shape(int bits, int gpr, int64_t n, int64_t d, int64_t T, int ntask) {
@@ -236,7 +259,8 @@ sk_status sk_linear_fwd(const void* packed, const uint16_t* lut, int bits, int g
   st = device_state(&check);
   if (st != SK_OK) return st;
   sk::Problem p = make_problem(packed, lut, bits, gpr, n, d, T, task, ntask, check);
-  cudaError_t e = sk::launch_gemv_fwd(p, X, Y, reinterpret_cast<cudaStream_t>(stream));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = use_tensor_cores_fwd(p) ? sk::launch_fwd_tc(p, X, Y, s) : sk::launch_gemv_fwd(p, X, Y, s);
   return e == cudaSuccess ? ok() : cuda_fail(e, "forward kernel launch");
 }
 

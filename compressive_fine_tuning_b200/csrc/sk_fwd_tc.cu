@@ -1,0 +1,350 @@
+// Forward of the sketched linear layer on the 5th-generation tensor cores:
+//   Y[t][i] = sum_j X[t][j] * Theta_hat[i][j]
+// ("SpaLLM: Unified Compressive Adaptation of LLMs with Sketching", section
+// 2.3: one compressed matmul per layer; Eq. 1 with groups per row gives
+// Theta_hat).
+//
+// The MMA computes the transposed tile Y^T[128 rows x N tokens] =
+// Theta_hat[128 x K] * X[N x K]^T with the dequantised weights as operand A in
+// tensor memory and the activations as operand B in shared memory:
+//   * TMA brings, per 128-column step, the packed index tile (128 rows) and
+//     the X tile (N tokens, two 64-column swizzled boxes) into shared memory;
+//   * eight dequantisation warps each own 32 weight rows (one per thread, the
+//     thread's row is its TMEM lane) and half of the step's columns; a thread
+//     looks its own row's indices up in register byte-plane LUTs and writes
+//     the bf16 weights straight into tensor memory (tcgen05.st), so the
+//     dequantised tile never touches shared memory;
+//   * one thread issues tcgen05.mma (kind::f16, A from TMEM, B from SMEM,
+//     fp32 accumulator in TMEM) and tcgen05.commit hands stages back;
+//   * the epilogue reads the accumulator with tcgen05.ld (thread = row) and
+//     writes bf16 Y.
+// Decode batches (N <= 64) are split along K over a thread-block cluster; the
+// partial accumulators are summed in a fixed order through distributed shared
+// memory, so the result is deterministic and needs no workspace.
+#include <cooperative_groups.h>
+
+#include "sk_tc.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace sk {
+namespace {
+
+constexpr int kDequantWarps = 8;
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 320;
+constexpr int KSTEP = 128;      // weight columns per pipeline step
+constexpr int SA = 2;           // tensor-memory stages of operand A
+constexpr int A_COLS = KSTEP / 2;  // 32-bit TMEM columns per A stage (bf16 pairs)
+
+__host__ __device__ constexpr int align1k(int x) { return (x + 1023) / 1024 * 1024; }
+__host__ __device__ constexpr int pow2ceil(int x) { int p = 32; while (p < x) p *= 2; return p; }
+
+template <int BITS, int N>
+struct Cfg {
+  static constexpr int S = N >= 256 ? 3 : (N >= 128 ? 5 : 6);  // shared-memory stages
+  static constexpr int KB = KSTEP * BITS / 8;                  // index bytes per row per step
+  static constexpr int X_BOX = N * 128;                        // one 64-column box of X
+  static constexpr int X_BYTES = 2 * X_BOX;
+  static constexpr int IDX_OFF = align1k(X_BYTES);
+  static constexpr int IDX_BYTES = 128 * KB;
+  static constexpr int STAGE = IDX_OFF + align1k(IDX_BYTES);
+  static constexpr int BAR_OFF = S * STAGE;
+  static constexpr int SMEM = 1024 + BAR_OFF + 256;            // + alignment slack + barriers
+  static constexpr int D_COL = SA * A_COLS;
+  static constexpr int TMEM_COLS = pow2ceil(D_COL + N);
+  static constexpr uint32_t IDESC = tc::idesc_bf16(128, N, 0, 0);
+  static_assert(N % 16 == 0 && N >= 16 && N <= 256, "UMMA N for M = 128");
+  static_assert(N * 128 * 4 <= BAR_OFF, "split-K partials reuse the stage memory");
+};
+
+struct FwdArgs {
+  const uint16_t* lut;
+  int64_t n, d, gs, T;
+  int gpr;
+  int steps_total;  // ceil(d / KSTEP)
+  uint16_t* Y;
+  unsigned int* check;
+};
+
+// The thread's two 32-column chunks of the step (half h of the 128 columns),
+// read from the TMA-swizzled index tile.
+template <int BITS>
+__device__ __forceinline__ void read_idx(const uint8_t* tile, int r, int h, Chunk<BITS> (&ch)[2]) {
+  if constexpr (BITS == 4) {         // 64-byte rows, 64B swizzle: chunk q at q ^ ((r >> 1) & 3)
+    const int sw = (r >> 1) & 3;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const uint4 v = *reinterpret_cast<const uint4*>(tile + r * 64 + 16 * ((2 * h + c) ^ sw));
+      ch[c].w[0] = v.x; ch[c].w[1] = v.y; ch[c].w[2] = v.z; ch[c].w[3] = v.w;
+    }
+  } else if constexpr (BITS == 2) {  // 32-byte rows, 32B swizzle: chunk q at q ^ ((r >> 2) & 1)
+    const uint4 v = *reinterpret_cast<const uint4*>(tile + r * 32 + 16 * (h ^ ((r >> 2) & 1)));
+    ch[0].w[0] = v.x; ch[0].w[1] = v.y; ch[1].w[0] = v.z; ch[1].w[1] = v.w;
+  } else {                           // 48-byte rows, no swizzle (conflict-free as is)
+    const uint2* p = reinterpret_cast<const uint2*>(tile + r * 48 + 24 * h);
+    const uint2 a = p[0], b = p[1], c = p[2];
+    ch[0].w[0] = a.x; ch[0].w[1] = a.y; ch[0].w[2] = b.x;
+    ch[1].w[0] = b.y; ch[1].w[1] = c.x; ch[1].w[2] = c.y;
+  }
+}
+
+template <int BITS, int N>
+__global__ void __launch_bounds__(kThreads, N <= 64 ? 2 : 1)
+fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_idx, FwdArgs a) {
+  using C = Cfg<BITS, N>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+  uint64_t* empty = full + C::S;
+  uint64_t* a_full = empty + C::S;
+  uint64_t* a_empty = a_full + SA;
+  uint64_t* d_full = a_empty + SA;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(d_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = tc::warp_id(), lane = tc::lane_id();
+  const int ks = blockIdx.x, ksplit = gridDim.x;
+  const int64_t m0 = (int64_t)blockIdx.y * 128;
+  const int t0 = blockIdx.z * N;
+  const int s0 = (int)((int64_t)ks * a.steps_total / ksplit);
+  const int s1 = (int)((int64_t)(ks + 1) * a.steps_total / ksplit);
+  const int nsteps = s1 - s0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::S; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], kDequantWarps + 1);
+    }
+    for (int i = 0; i < SA; ++i) {
+      tc::mbar_init(&a_full[i], kDequantWarps);
+      tc::mbar_init(&a_empty[i], 1);
+    }
+    tc::mbar_init(d_full, 1);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == kMmaWarp) tc::tmem_alloc(tmem_slot, C::TMEM_COLS);
+  if (warp == kTmaWarp && lane == 0) {
+    tc::tma_prefetch(&tm_x);
+    tc::tma_prefetch(&tm_idx);
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kTmaWarp) {
+    // ---------------- producer: TMA loads ----------------
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < nsteps && !*abort_flag; ++i) {
+        const int s = i % C::S;
+        if (!tc::mbar_wait(&empty[s], ((i / C::S) & 1) ^ 1, a.check)) { *abort_flag = 1; break; }
+        uint8_t* st = smem + s * C::STAGE;
+        tc::mbar_arrive_expect_tx(&full[s], C::X_BYTES + C::IDX_BYTES);
+        const int k0 = (s0 + i) * KSTEP;
+        tc::tma_load_2d(st, &tm_x, &full[s], k0, t0);
+        tc::tma_load_2d(st + C::X_BOX, &tm_x, &full[s], k0 + 64, t0);
+        tc::tma_load_2d(st + C::IDX_OFF, &tm_idx, &full[s], (s0 + i) * C::KB, (int)m0);
+        ++issued;
+      }
+      // never leave with a copy still landing in shared memory
+      for (int j = issued > C::S ? issued - C::S : 0; j < issued; ++j)
+        tc::mbar_wait(&full[j % C::S], (j / C::S) & 1, a.check);
+    }
+  } else if (warp == kMmaWarp) {
+    // ---------------- MMA issue ----------------
+    if (lane == 0) {
+      bool ok = true;
+      for (int i = 0; i < nsteps; ++i) {
+        const int s = i % C::S, ai = i % SA;
+        if (*abort_flag || !tc::mbar_wait(&full[s], (i / C::S) & 1, a.check) ||
+            !tc::mbar_wait(&a_full[ai], (i / SA) & 1, a.check)) {
+          *abort_flag = 1; ok = false; break;
+        }
+        tc::tc_fence_after();
+        const uint32_t xb = tc::smem_u32(smem + s * C::STAGE);
+#pragma unroll
+        for (int kk = 0; kk < KSTEP / 16; ++kk) {
+          const uint64_t bd = tc::sdesc(xb + (kk >> 2) * C::X_BOX + (kk & 3) * 32, 16, 1024, tc::kSwizzle128);
+          tc::mma_ts(tmem + C::D_COL, tmem + ai * A_COLS + kk * 8, bd, C::IDESC, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc::mma_commit(&empty[s]);
+        tc::mma_commit(&a_empty[ai]);
+      }
+      if (ok) tc::mma_commit(d_full);
+    }
+  } else {
+    // ---------------- dequantisation into tensor memory ----------------
+    const int quad = warp & 3, h = warp >> 2;
+    const int r = quad * 32 + lane;
+    const int64_t row = m0 + r;
+    const bool row_ok = row < a.n;
+    const uint16_t* lut_row = a.lut + (row_ok ? row : 0) * a.gpr * (1 << BITS);
+    int64_t cur_g = -1;
+    LutRegs<BITS> L;
+    for (int i = 0; i < nsteps; ++i) {
+      const int s = i % C::S, ai = i % SA;
+      if (*abort_flag || !tc::mbar_wait(&full[s], (i / C::S) & 1, a.check) ||
+          !tc::mbar_wait(&a_empty[ai], ((i / SA) & 1) ^ 1, a.check)) {
+        *abort_flag = 1; break;
+      }
+      tc::tc_fence_after();
+      Chunk<BITS> ch[2];
+      read_idx<BITS>(smem + s * C::STAGE + C::IDX_OFF, r, h, ch);
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&empty[s]);
+      uint32_t v[32];
+      const int64_t col0 = (int64_t)(s0 + i) * KSTEP + h * 64;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int64_t col = col0 + 32 * c;
+        if (row_ok && col < a.d) {
+          const int64_t g = col / a.gs;
+          if (g != cur_g) {
+            load_lut<BITS>(lut_row + g * (1 << BITS), L);
+            cur_g = g;
+          }
+          uint32_t o[16];
+          dequant_chunk<BITS>(ch[c], L, o);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[16 * c + e] = o[e];
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[16 * c + e] = 0u;
+        }
+      }
+      tc::tmem_st32(tc::tmem_addr(tmem, quad * 32, ai * A_COLS + h * 32), v);
+      tc::tmem_st_wait();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&a_full[ai]);
+    }
+  }
+
+  // ---------------- epilogue ----------------
+  __syncthreads();
+  const bool aborted = *abort_flag != 0;
+  float* red = reinterpret_cast<float*>(smem);  // [N][128] partial sums (split-K)
+  if (warp < kDequantWarps) {
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const int64_t row = m0 + r;
+    if (!aborted && tc::mbar_wait(d_full, 0, a.check)) {
+      tc::tc_fence_after();
+      // warps w and w + 4 share a lane quadrant and split the N columns
+      constexpr int GROUPS = N / 16;
+      for (int gi = warp >> 2; gi < GROUPS; gi += 2) {
+        uint32_t v[16];
+        tc::tmem_ld16(tc::tmem_addr(tmem, quad * 32, C::D_COL + gi * 16), v);
+        tc::tmem_ld_wait();
+        if (ksplit == 1) {
+          if (row < a.n) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int64_t t = t0 + gi * 16 + j;
+              if (t < a.T) {
+                __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(v[j]));
+                a.Y[t * a.n + row] = *reinterpret_cast<uint16_t*>(&b);
+              }
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) red[(gi * 16 + j) * 128 + r] = __uint_as_float(v[j]);
+        }
+      }
+    } else if (ksplit > 1) {
+      for (int j = 0; j < N; ++j) red[j * 128 + r] = 0.f;
+    }
+  }
+  if (ksplit > 1) {
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    // CTA `ks` of the cluster sums rows [ks * 128 / ksplit, (ks + 1) * 128 / ksplit)
+    const int rows_per = 128 / ksplit;
+    for (int e = threadIdx.x; e < N * rows_per; e += kThreads) {
+      const int t = e / rows_per, rr = ks * rows_per + e % rows_per;
+      float sum = 0.f;
+      for (int q = 0; q < ksplit; ++q) sum += cluster.map_shared_rank(red, q)[t * 128 + rr];
+      const int64_t tg = t0 + t, row = m0 + rr;
+      if (tg < a.T && row < a.n) {
+        __nv_bfloat16 b = __float2bfloat16_rn(sum);
+        a.Y[tg * a.n + row] = *reinterpret_cast<uint16_t*>(&b);
+      }
+    }
+    cluster.sync();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int BITS, int N>
+cudaError_t launch_n(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStream_t s) {
+  using C = Cfg<BITS, N>;
+  cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<BITS, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  CUtensorMap tm_x, tm_idx;
+  e = make_tmap_2d(&tm_x, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)p.d, (uint64_t)p.T,
+                               (uint64_t)p.d * 2, 64, N, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
+  const CUtensorMapSwizzle isw = BITS == 4 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                 : BITS == 2 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_NONE;
+  e = make_tmap_2d(&tm_idx, p.packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)p.row_bytes, (uint64_t)p.n,
+                   (uint64_t)p.row_bytes, C::KB, 128, isw);
+  if (e != cudaSuccess) return e;
+
+  const int steps = (int)((p.d + KSTEP - 1) / KSTEP);
+  const int64_t m_blocks = (p.n + 127) / 128;
+  const int64_t t_tiles = (p.T + N - 1) / N;
+  int ksplit = 1;
+  if (N <= 64) {
+    const int64_t target = 2 * (int64_t)num_sms();
+    while (ksplit < 8 && m_blocks * t_tiles * ksplit * 2 <= target && ksplit * 2 <= steps) ksplit *= 2;
+  }
+  FwdArgs args{p.lut, p.n, p.d, p.gs, p.T, p.gpr, steps, Y, p.check};
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)ksplit, (unsigned)m_blocks, (unsigned)t_tiles);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = ksplit;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fwd_tc_kernel<BITS, N>, tm_x, tm_idx, args);
+}
+
+template <int BITS>
+cudaError_t launch_bits(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStream_t s) {
+  if (p.T <= 16) return launch_n<BITS, 16>(p, X, Y, s);
+  if (p.T <= 32) return launch_n<BITS, 32>(p, X, Y, s);
+  if (p.T <= 64) return launch_n<BITS, 64>(p, X, Y, s);
+  if (p.T <= 128) return launch_n<BITS, 128>(p, X, Y, s);
+  return launch_n<BITS, 256>(p, X, Y, s);
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_tc(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStream_t s) {
+  cudaError_t e;
+  switch (p.bits) {
+    case 2: e = launch_bits<2>(p, X, Y, s); break;
+    case 3: e = launch_bits<3>(p, X, Y, s); break;
+    default: e = launch_bits<4>(p, X, Y, s); break;
+  }
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace sk

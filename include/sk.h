@@ -77,6 +77,8 @@ typedef enum {
 /* Device check word bits (sk_device_check). */
 #define SK_CHECK_TASK_RANGE 1u   /* a task id outside [0, ntask) was seen      */
 #define SK_CHECK_INDEX_RANGE 2u  /* sk_pack saw an index >= 2^bits             */
+#define SK_CHECK_TIMEOUT 4u      /* a kernel gave up waiting on its own pipeline
+                                    (an internal error; its outputs are invalid) */
 
 /* Operation selectors for sk_workspace_bytes. */
 #define SK_OP_FWD 0

@@ -261,3 +261,43 @@ def test_llama7b_decode_full_size_sampled(layer, T):
     Y = sk.linear_fwd(packed, lut, c.bits, X)
     rows = np.sort(synth.rng_for(8100 + layer).choice(n, size=96, replace=False))
     gc.check_fwd(c, Y, rows=rows)
+
+
+# ---------------------------------------------------------------------------
+# both forward kernels at every batch size (SK_FWD_PATH forces one of them)
+# ---------------------------------------------------------------------------
+
+@pytest.fixture
+def fwd_path(monkeypatch):
+    def set_path(p):
+        monkeypatch.setenv("SK_FWD_PATH", p)
+    yield set_path
+
+
+@pytest.mark.parametrize("path", ["tc", "gemv"])
+@pytest.mark.parametrize("shape", [(256, 512, 4, 1), (136, 320, 2, 5), (264, 1376, 3, 1), (1024, 4096, 4, 8)])
+@pytest.mark.parametrize("T", [1, 2, 17, 64, 129])
+def test_forward_each_path(fwd_path, path, shape, T):
+    sk = _sk()
+    fwd_path(path)
+    c = _case(shape, T, 9000 + T)
+    packed, lut, X, dY, task = gc.dev_case(c)
+    Y = sk.linear_fwd(packed, lut, c.bits, X, task)
+    gc.check_fwd(c, Y)
+    assert sk.device_check() == 0
+
+
+@pytest.mark.parametrize("T", [1, 16])
+def test_identity_exact_tc_path(fwd_path, T):
+    sk = _sk()
+    fwd_path("tc")
+    n = 1024
+    rng = synth.rng_for(9100 + T)
+    idx = torch.eye(n, dtype=torch.uint8, device="cuda")
+    packed = sk.pack(idx, 2)
+    lut = torch.full((1, n, 1, 4), float("nan"), dtype=torch.float16, device="cuda")
+    lut[..., 0] = 0.0
+    lut[..., 1] = 1.0
+    X = torch.from_numpy(synth.make_bf16(rng, (T, n), 1.0).view(np.int16)).cuda().view(torch.bfloat16)
+    Y = sk.linear_fwd(packed, lut, 2, X)
+    assert torch.equal(Y.view(torch.int16), X.view(torch.int16))
