@@ -68,6 +68,9 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--launch-events", choices=("auto", "on", "off"), default="auto",
+                    help="capture timing events between launches (per-kernel durations; they add "
+                         "a few microseconds per launch); auto = only when a step mixes kernels")
     return ap.parse_args()
 
 
@@ -277,6 +280,8 @@ def run_ours(args, w, rank, world, device):
 
     stream = torch.cuda.Stream(device)
     K, W = args.steps, args.warmup
+    if args.launch_events == "auto":
+        args.launch_events = "off" if len(w["ops"]) == 1 else "on"
 
     # warm-up (eager), also the first-call setup of every kernel
     with torch.cuda.stream(stream):
@@ -291,10 +296,12 @@ def run_ours(args, w, rank, world, device):
         g = torch.cuda.CUDAGraph()
         evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(plan) + 1)]
         with torch.cuda.graph(g, stream=stream):
-            evs[0].record()
+            if args.launch_events == "on":
+                evs[0].record()
             for j, (li, T, op, u) in enumerate(plan):
                 launch(li, T, op, W + s)
-                evs[j + 1].record()
+                if args.launch_events == "on":
+                    evs[j + 1].record()
         graphs.append(g)
         ev.append(evs)
     torch.cuda.synchronize(device)
@@ -325,9 +332,14 @@ def run_ours(args, w, rank, world, device):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
 
-    # per-launch durations from the captured events
-    per_launch = np.array([[ev[s][j].elapsed_time(ev[s][j + 1]) for j in range(len(plan))] for s in range(K)])
-    launches_ms = per_launch.sum(axis=0) / K  # mean per launch position
+    # per-launch durations from the captured events (without them: the step
+    # time spread over the launches in proportion to their units)
+    if args.launch_events == "on":
+        per_launch = np.array([[ev[s][j].elapsed_time(ev[s][j + 1]) for j in range(len(plan))] for s in range(K)])
+        launches_ms = per_launch.sum(axis=0) / K  # mean per launch position
+    else:
+        u = np.array([p[3] for p in plan], dtype=np.float64)
+        launches_ms = (ms / K) * u / u.sum()
 
     total_units = step_units * K * world
     value = total_units / (ms / 1e3)

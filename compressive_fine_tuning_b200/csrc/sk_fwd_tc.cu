@@ -35,7 +35,6 @@ constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kThreads = 320;
 constexpr int KSTEP = 128;      // weight columns per pipeline step
-constexpr int SA = 2;           // tensor-memory stages of operand A
 constexpr int A_COLS = KSTEP / 2;  // 32-bit TMEM columns per A stage (bf16 pairs)
 
 __host__ __device__ constexpr int align1k(int x) { return (x + 1023) / 1024 * 1024; }
@@ -43,7 +42,10 @@ __host__ __device__ constexpr int pow2ceil(int x) { int p = 32; while (p < x) p 
 
 template <int BITS, int N>
 struct Cfg {
-  static constexpr int S = N >= 256 ? 3 : (N >= 128 ? 5 : 6);  // shared-memory stages
+  // decode tiles (N <= 64) keep under half of an SM's shared and tensor memory
+  // so that the next launch's CTA can share the SM (programmatic dependent launch)
+  static constexpr int S = N >= 256 ? 3 : N >= 128 ? 5 : N >= 64 ? 4 : N >= 32 ? 6 : 8;  // shared-memory stages
+  static constexpr int SA = N <= 64 ? 3 : 2;                   // tensor-memory stages of operand A
   static constexpr int KB = KSTEP * BITS / 8;                  // index bytes per row per step
   static constexpr int X_BOX = N * 128;                        // one 64-column box of X
   static constexpr int X_BYTES = 2 * X_BOX;
@@ -53,10 +55,12 @@ struct Cfg {
   static constexpr int BAR_OFF = S * STAGE;
   static constexpr int SMEM = 1024 + BAR_OFF + 256;            // + alignment slack + barriers
   static constexpr int D_COL = SA * A_COLS;
+  static constexpr int ROWS_PER_RANK_MAX = 128;
   static constexpr int TMEM_COLS = pow2ceil(D_COL + N);
   static constexpr uint32_t IDESC = tc::idesc_bf16(128, N, 0, 0);
   static_assert(N % 16 == 0 && N >= 16 && N <= 256, "UMMA N for M = 128");
   static_assert(N * 128 * 4 <= BAR_OFF, "split-K partials reuse the stage memory");
+  static_assert(SA * A_COLS + N <= TMEM_COLS, "tensor memory budget");
 };
 
 struct FwdArgs {
@@ -99,6 +103,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* empty = full + C::S;
   uint64_t* a_full = empty + C::S;
+  // let the next launch in the stream start its prologue while this one runs
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  constexpr int SA = C::SA;
   uint64_t* a_empty = a_full + SA;
   uint64_t* d_full = a_empty + SA;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(d_full + 1);
@@ -134,6 +141,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // inputs may come from the previous launch: wait for it before reading any
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == kTmaWarp) {
     // ---------------- producer: TMA loads ----------------
@@ -183,9 +192,16 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
     const int64_t row = m0 + r;
     const bool row_ok = row < a.n;
     const uint16_t* lut_row = a.lut + (row_ok ? row : 0) * a.gpr * (1 << BITS);
-    int64_t cur_g = -1;
+    // group bookkeeping in 32-bit arithmetic, advanced incrementally (no divisions in the loop)
+    const int d32 = (int)a.d, gs32 = (int)a.gs;
+    int col = s0 * KSTEP + h * 64;          // first column of this thread's half of the step
+    int g = col / gs32;
+    if (g >= a.gpr) g = a.gpr - 1;
+    int g_end = (g + 1) * gs32;             // first column past group g
+    // fetch the first group's table now, overlapping the first TMA round trip
     LutRegs<BITS> L;
-    for (int i = 0; i < nsteps; ++i) {
+    load_lut<BITS>(lut_row + g * (1 << BITS), L);
+    for (int i = 0; i < nsteps; ++i, col += KSTEP) {
       const int s = i % C::S, ai = i % SA;
       if (*abort_flag || !tc::mbar_wait(&full[s], (i / C::S) & 1, a.check) ||
           !tc::mbar_wait(&a_empty[ai], ((i / SA) & 1) ^ 1, a.check)) {
@@ -197,15 +213,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&empty[s]);
       uint32_t v[32];
-      const int64_t col0 = (int64_t)(s0 + i) * KSTEP + h * 64;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        const int64_t col = col0 + 32 * c;
-        if (row_ok && col < a.d) {
-          const int64_t g = col / a.gs;
-          if (g != cur_g) {
+        const int cc = col + 32 * c;
+        if (row_ok && cc < d32) {
+          if (cc >= g_end) {             // a chunk never straddles groups (gs % 32 == 0)
+            do { ++g; g_end += gs32; } while (cc >= g_end);
             load_lut<BITS>(lut_row + g * (1 << BITS), L);
-            cur_g = g;
           }
           uint32_t o[16];
           dequant_chunk<BITS>(ch[c], L, o);
@@ -227,55 +241,62 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
   // ---------------- epilogue ----------------
   __syncthreads();
   const bool aborted = *abort_flag != 0;
-  float* red = reinterpret_cast<float*>(smem);  // [N][128] partial sums (split-K)
+  // split-K: rows [q * rows_per, (q + 1) * rows_per) of every CTA's partial go
+  // to cluster rank q, slot = the sender's rank; layout [slot][N][rows_per]
+  const int rows_per = 128 / ksplit;
+  float* inbox = reinterpret_cast<float*>(smem);
+  cg::cluster_group cluster = cg::this_cluster();
+  // the accumulator is final once d_full fires; the tensor cores have then also
+  // finished reading this CTA's stage memory, which becomes the split-K inbox
+  const bool have = warp < kDequantWarps && !aborted && tc::mbar_wait(d_full, 0, a.check);
+  if (have) tc::tc_fence_after();
+  if (ksplit > 1) cluster.sync();  // every peer's stage memory is free now
   if (warp < kDequantWarps) {
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const int64_t row = m0 + r;
-    if (!aborted && tc::mbar_wait(d_full, 0, a.check)) {
-      tc::tc_fence_after();
-      // warps w and w + 4 share a lane quadrant and split the N columns
-      constexpr int GROUPS = N / 16;
-      for (int gi = warp >> 2; gi < GROUPS; gi += 2) {
-        uint32_t v[16];
+    constexpr int GROUPS = N / 16;
+    // warps w and w + 4 share a lane quadrant and split the N columns
+    for (int gi = warp >> 2; gi < GROUPS; gi += 2) {
+      uint32_t v[16];
+      if (have) {
         tc::tmem_ld16(tc::tmem_addr(tmem, quad * 32, C::D_COL + gi * 16), v);
         tc::tmem_ld_wait();
-        if (ksplit == 1) {
-          if (row < a.n) {
+      } else {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int64_t t = t0 + gi * 16 + j;
-              if (t < a.T) {
-                __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(v[j]));
-                a.Y[t * a.n + row] = *reinterpret_cast<uint16_t*>(&b);
-              }
+        for (int j = 0; j < 16; ++j) v[j] = 0u;
+      }
+      if (ksplit == 1) {
+        if (row < a.n) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int64_t t = t0 + gi * 16 + j;
+            if (t < a.T) {
+              __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(v[j]));
+              a.Y[t * a.n + row] = *reinterpret_cast<uint16_t*>(&b);
             }
           }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) red[(gi * 16 + j) * 128 + r] = __uint_as_float(v[j]);
         }
+      } else {
+        const int q = r / rows_per, rr = r % rows_per;
+        float* dst = cluster.map_shared_rank(inbox, q) + (ks * N + gi * 16) * rows_per + rr;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) dst[j * rows_per] = __uint_as_float(v[j]);
       }
-    } else if (ksplit > 1) {
-      for (int j = 0; j < N; ++j) red[j * 128 + r] = 0.f;
     }
   }
   if (ksplit > 1) {
-    cg::cluster_group cluster = cg::this_cluster();
-    cluster.sync();
-    // CTA `ks` of the cluster sums rows [ks * 128 / ksplit, (ks + 1) * 128 / ksplit)
-    const int rows_per = 128 / ksplit;
+    cluster.sync();  // all pushes landed
     for (int e = threadIdx.x; e < N * rows_per; e += kThreads) {
-      const int t = e / rows_per, rr = ks * rows_per + e % rows_per;
+      const int t = e / rows_per, rr = e % rows_per;
       float sum = 0.f;
-      for (int q = 0; q < ksplit; ++q) sum += cluster.map_shared_rank(red, q)[t * 128 + rr];
-      const int64_t tg = t0 + t, row = m0 + rr;
+      for (int q = 0; q < ksplit; ++q) sum += inbox[(q * N + t) * rows_per + rr];
+      const int64_t tg = t0 + t, row = m0 + ks * rows_per + rr;
       if (tg < a.T && row < a.n) {
         __nv_bfloat16 b = __float2bfloat16_rn(sum);
         a.Y[tg * a.n + row] = *reinterpret_cast<uint16_t*>(&b);
       }
     }
-    cluster.sync();
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -307,6 +328,8 @@ cudaError_t launch_n(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStrea
   if (N <= 64) {
     const int64_t target = 2 * (int64_t)num_sms();
     while (ksplit < 8 && m_blocks * t_tiles * ksplit * 2 <= target && ksplit * 2 <= steps) ksplit *= 2;
+    const int forced = env_int("SK_TC_KSPLIT", 0);
+    if (forced == 1 || forced == 2 || forced == 4 || forced == 8) ksplit = forced <= steps ? forced : 1;
   }
   FwdArgs args{p.lut, p.n, p.d, p.gs, p.T, p.gpr, steps, Y, p.check};
 
@@ -315,13 +338,15 @@ cudaError_t launch_n(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStrea
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = ksplit;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, fwd_tc_kernel<BITS, N>, tm_x, tm_idx, args);
 }
 

@@ -4,9 +4,9 @@
 // Table 5: decode is where the single-tower layer pays off).
 //
 // Work split: a warp owns R weight rows and splits their columns across its
-// lanes; each lane walks pairs of 32-column chunks (one 16/8/12-byte index
-// load per chunk, consecutive lanes on consecutive chunks so a warp-wide load
-// is one contiguous span of the row), dequantises them through register LUTs
+// lanes; each lane walks 32-column chunks (one 16/8/12-byte index load per
+// chunk, consecutive lanes on consecutive chunks so a warp-wide load is one
+// contiguous span of the row), dequantises them through register LUTs
 // and accumulates R x TT fp32 dot products with bf16 x fp32 fused multiply-adds.
 // A warp-shuffle tree then reduces the lane partial sums.  Tokens are taken TT
 // at a time; tokens with different LUT sets re-dequantise the chunk.
@@ -20,6 +20,8 @@ constexpr int kWarps = 4;
 template <int BITS, int R, int TT>
 __global__ void __launch_bounds__(kWarps * 32) gemv_fwd_kernel(Problem p, const uint16_t* __restrict__ X,
                                                                uint16_t* __restrict__ Y) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // inputs may come from the previous launch
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row0 = ((int64_t)blockIdx.x * kWarps + warp) * R;
   if (row0 >= p.n) return;
@@ -41,8 +43,10 @@ __global__ void __launch_bounds__(kWarps * 32) gemv_fwd_kernel(Problem p, const 
 #pragma unroll
       for (int u = 0; u < TT; ++u) acc[r][u] = 0.f;
 
-    for (int64_t c = lane; c < chunks; c += 32) {
-      const int64_t g = c / cpg;
+    const int cpg32 = (int)cpg;
+    int g = lane / cpg32, g_next = (g + 1) * cpg32;   // chunk group, advanced without divisions
+    for (int c = lane; c < (int)chunks; c += 32) {
+      while (c >= g_next) { ++g; g_next += cpg32; }
       Chunk<BITS> ch[R];
 #pragma unroll
       for (int r = 0; r < R; ++r) ch[r] = load_chunk<BITS>(rows[r], c);
@@ -105,9 +109,17 @@ __global__ void __launch_bounds__(kWarps * 32) gemv_fwd_kernel(Problem p, const 
 template <int BITS, int R, int TT>
 cudaError_t launch(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStream_t s) {
   const int64_t rows_per_cta = (int64_t)kWarps * R;
-  const unsigned grid = (unsigned)((p.n + rows_per_cta - 1) / rows_per_cta);
-  gemv_fwd_kernel<BITS, R, TT><<<grid, kWarps * 32, 0, s>>>(p, X, Y);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((p.n + rows_per_cta - 1) / rows_per_cta), 1, 1);
+  cfg.blockDim = dim3(kWarps * 32, 1, 1);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_fwd_kernel<BITS, R, TT>, p, X, Y);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <int BITS>

@@ -264,6 +264,11 @@ __device__ __forceinline__ const uint16_t* lut_ptr(const Problem& p, int tau, in
   return p.lut + (((int64_t)tau * p.n + i) * p.gpr + g) * (1 << p.bits);
 }
 
+// Host-side knobs read from the environment (experiments and tests).
+int env_int(const char* name, int dflt);
+// Programmatic dependent launch for the forward kernels (SK_PDL=0 turns it off).
+bool pdl_enabled();
+
 // Host-side launchers (one per kernel file).  They return cudaGetLastError().
 cudaError_t launch_pack(const uint8_t* idx, int64_t n, int64_t d, int bits, uint8_t* packed,
                         int64_t row_bytes, unsigned int* check, cudaStream_t s);

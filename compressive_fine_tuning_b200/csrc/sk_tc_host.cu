@@ -3,6 +3,7 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <cstdlib>
 #include <mutex>
 
 #include "sk_tc.cuh"
@@ -41,6 +42,14 @@ cudaError_t make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
+
+int env_int(const char* name, int dflt) {
+  const char* v = getenv(name);
+  if (v == nullptr || *v == 0) return dflt;
+  return atoi(v);
+}
+
+bool pdl_enabled() { return env_int("SK_PDL", 1) != 0; }
 
 int num_sms() {
   int dev = 0;
