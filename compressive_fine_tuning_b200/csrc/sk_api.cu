@@ -96,6 +96,19 @@ int env_path(const char* name) {
   return 0;
 }
 
+// Backward kernel choice: the tensor-core kernels take single-LUT-set batches
+// of at least kBwdTcMinT tokens on layers with n, d >= 64; SK_BWD_PATH=simt|tc
+// forces a path.  sk_workspace_bytes uses the same rule.
+constexpr int64_t kBwdTcMinT = 64;
+
+bool use_tensor_cores_bwd(int64_t n, int64_t d, int64_t T, int ntask) {
+  const bool tc_ok = ntask == 1 && n >= 64 && d >= 64;
+  const int forced = env_path("SK_BWD_PATH");
+  if (forced == 1) return false;
+  if (forced == 2) return tc_ok;
+  return tc_ok && T >= kBwdTcMinT;
+}
+
 bool use_tensor_cores_fwd(const sk::Problem& p) {
   const bool tc_ok = (p.task == nullptr || p.ntask == 1) && p.d >= 128;
   const int forced = env_path("SK_FWD_PATH");
@@ -220,8 +233,10 @@ sk_status sk_dequant(const void* packed, const uint16_t* lut, int bits, int gpr,
 }
 
 size_t sk_workspace_bytes(int op, int64_t n, int64_t d, int bits, int gpr, int64_t T, int ntask) {
-  (void)n; (void)d; (void)bits; (void)gpr; (void)T; (void)ntask;
   if (op < SK_OP_FWD || op > SK_OP_BWD_LUT) return 0;
+  if (bits < 2 || bits > 4 || n < 1 || d < 32 || gpr < 1 || d % gpr != 0 || T < 1) return 0;
+  if (op == SK_OP_BWD_LUT && use_tensor_cores_bwd(n, d, T, ntask))
+    return sk::dlut_tc_workspace(n, d, bits, gpr);
   return 0;
 }
 
@@ -281,7 +296,9 @@ sk_status sk_linear_bwd_input(const void* packed, const uint16_t* lut, int bits,
   st = device_state(&check);
   if (st != SK_OK) return st;
   sk::Problem p = make_problem(packed, lut, bits, gpr, n, d, T, task, ntask, check);
-  cudaError_t e = sk::launch_simt_bwd_input(p, dY, dX, reinterpret_cast<cudaStream_t>(stream));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = use_tensor_cores_bwd(n, d, T, ntask) ? sk::launch_dx_tc(p, dY, dX, s)
+                                                                          : sk::launch_simt_bwd_input(p, dY, dX, s);
   return e == cudaSuccess ? ok() : cuda_fail(e, "input-gradient kernel launch");
 }
 
@@ -310,7 +327,16 @@ sk_status sk_linear_bwd_lut(const void* packed, int bits, int gpr, int64_t n, in
   st = device_state(&check);
   if (st != SK_OK) return st;
   sk::Problem p = make_problem(packed, nullptr, bits, gpr, n, d, T, task, ntask, check);
-  cudaError_t e = sk::launch_simt_bwd_lut(p, X, dY, dlut, accumulate, reinterpret_cast<cudaStream_t>(stream));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (use_tensor_cores_bwd(n, d, T, ntask)) {
+    const size_t need = sk::dlut_tc_workspace(n, d, bits, gpr);
+    if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))
+      return fail(SK_ERR_INVALID_ARG, "workspace of %zu bytes (16-byte aligned) required", need);
+    e = sk::launch_dlut_tc(p, X, dY, dlut, accumulate, workspace, s);
+  } else {
+    e = sk::launch_simt_bwd_lut(p, X, dY, dlut, accumulate, s);
+  }
   return e == cudaSuccess ? ok() : cuda_fail(e, "LUT-gradient kernel launch");
 }
 

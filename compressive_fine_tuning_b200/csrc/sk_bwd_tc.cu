@@ -1,0 +1,493 @@
+// Backward of the sketched linear layer on the 5th-generation tensor cores.
+//
+// Input gradient (chain rule through the frozen sketch):
+//   dX[t][j] = sum_i dY[t][i] * Theta_hat[i][j]
+// computed as the transposed tile dX^T[128 columns j x 256 tokens]:
+//   * operand A = Theta_hat^T (M = j, K = i) lives in shared memory in the
+//     MN-major 128-byte-swizzled layout; eight producer warps dequantise it,
+//     each thread owning one weight row i of the step (so the row's LUT is a
+//     register table) and one 32-column chunk, writing 16-byte swizzled stores;
+//   * operand B = dY (N = t, K = i) arrives by TMA (K-major, 128B swizzle);
+//   * one thread issues tcgen05.mma, the fp32 accumulator lives in TMEM, and
+//     the epilogue writes bf16 dX.
+//
+// LUT gradient (the corrected Eq. 6 of the "Sketch to Adapt" OpenReview
+// discussion, reply Q1): dlut[i][g][c] = sum_{j in g, idx[i][j] = c} (dY^T X)[i][j].
+//   * G tile [128 rows i x 256 columns j] = dY^T X over K = tokens, both
+//     operands MN-major straight from TMA;
+//   * the epilogue never writes G: each thread takes its row's accumulator
+//     32 columns at a time (tcgen05.ld), looks the indices up and adds every
+//     value into the (group, centroid) bin it selects.  Bins live in shared
+//     memory as [k][thread] (the dynamic bin index never causes a bank
+//     conflict); on a group change the thread writes its k sums as one
+//     partial for (column tile, row, group slot);
+//   * a second small kernel adds the partials of every group over the column
+//     tiles in a fixed order, so the result is deterministic, and writes or
+//     accumulates dlut.
+#include "sk_tc.cuh"
+
+namespace sk {
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
+
+__host__ __device__ constexpr int ceil_div(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
+
+// ============================================================================
+// dX
+// ============================================================================
+
+namespace dx {
+constexpr int N = 256;          // tokens per tile
+constexpr int KS = 64;          // weight rows (K) per pipeline step
+constexpr int S = 4;            // stages
+constexpr int B_BYTES = N * 128;             // dY tile: N rows x 64 bf16
+constexpr int A_BYTES = 2 * 8 * 1024;        // two 64-column MN atoms x 8 K-groups
+constexpr int STAGE = B_BYTES + A_BYTES;
+constexpr int BAR_OFF = S * STAGE;
+constexpr int SMEM = 1024 + BAR_OFF + 256;
+constexpr uint32_t IDESC = tc::idesc_bf16(128, N, /*a MN-major*/ 1, /*b K-major*/ 0);
+constexpr int TMEM_COLS = 256;
+}  // namespace dx
+
+struct DxArgs {
+  const uint8_t* packed;
+  int64_t row_bytes;
+  const uint16_t* lut;
+  int64_t n, d, gs, T;
+  int gpr;
+  uint16_t* dX;
+  unsigned int* check;
+};
+
+template <int BITS>
+__global__ void __launch_bounds__(kThreads, 1)
+dx_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, DxArgs a) {
+  using namespace dx;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full_b = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
+  uint64_t* full_a = full_b + S;
+  uint64_t* empty = full_a + S;
+  uint64_t* d_full = empty + S;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(d_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = tc::warp_id(), lane = tc::lane_id();
+  const int64_t j0 = (int64_t)blockIdx.x * 128;
+  const int t0 = blockIdx.y * N;
+  const int nsteps = ceil_div(a.n, KS);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      tc::mbar_init(&full_b[s], 1);
+      tc::mbar_init(&full_a[s], 8);
+      tc::mbar_init(&empty[s], 1);
+    }
+    tc::mbar_init(d_full, 1);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == kMmaWarp) tc::tmem_alloc(tmem_slot, TMEM_COLS);
+  if (warp == kTmaWarp && lane == 0) tc::tma_prefetch(&tm_dy);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kTmaWarp) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < nsteps && !*abort_flag; ++i) {
+        const int s = i % S;
+        if (!tc::mbar_wait(&empty[s], ((i / S) & 1) ^ 1, a.check)) { *abort_flag = 1; break; }
+        tc::mbar_arrive_expect_tx(&full_b[s], B_BYTES);
+        tc::tma_load_2d(smem + s * STAGE, &tm_dy, &full_b[s], i * KS, t0);
+        ++issued;
+      }
+      for (int j = issued > S ? issued - S : 0; j < issued; ++j) tc::mbar_wait(&full_b[j % S], (j / S) & 1, a.check);
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      bool ok = true;
+      for (int i = 0; i < nsteps; ++i) {
+        const int s = i % S;
+        if (*abort_flag || !tc::mbar_wait(&full_b[s], (i / S) & 1, a.check) ||
+            !tc::mbar_wait(&full_a[s], (i / S) & 1, a.check)) {
+          *abort_flag = 1; ok = false; break;
+        }
+        tc::tc_fence_after();
+        const uint32_t bb = tc::smem_u32(smem + s * STAGE);
+        const uint32_t ab = bb + B_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < KS / 16; ++kk) {
+          const uint64_t ad = tc::sdesc(ab + kk * 2048, 8192, 1024, tc::kSwizzle128);
+          const uint64_t bd = tc::sdesc(bb + kk * 32, 16, 1024, tc::kSwizzle128);
+          tc::mma_ss(tmem, ad, bd, IDESC, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc::mma_commit(&empty[s]);
+      }
+      if (ok) tc::mma_commit(d_full);
+    }
+  } else {
+    // producers: warp w fills K-group w (8 rows) of the A tile; lane = (chunk h, row r8)
+    const int r8 = lane & 7, h = lane >> 3;
+    const int lr = 8 * warp + r8;                    // row within the step
+    const int64_t j = j0 + 32 * h;                   // first column of this thread's chunk
+    const bool col_ok = j < a.d;
+    const int64_t cchunk = j >> 5;
+    const int64_t g = col_ok ? j / a.gs : 0;
+    const int m_atom = h >> 1;
+    // swizzled 16-byte slots of this thread's four chunks within the K-row
+    uint32_t slot_off[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) slot_off[q] = m_atom * 8192 + warp * 1024 + r8 * 128 + (((4 * (h & 1) + q) ^ r8) << 4);
+    // software pipeline: this step's index chunk and raw LUT entries are loaded one step ahead
+    Chunk<BITS> ch_next{};
+    uint4 lraw_next[2] = {};
+    auto fetch = [&](int i) {
+      const int64_t row = (int64_t)i * KS + lr;
+      if (col_ok && row < a.n) {
+        ch_next = load_chunk<BITS>(a.packed + row * a.row_bytes, cchunk);
+        const uint16_t* lp = a.lut + (row * a.gpr + g) * (1 << BITS);
+        if constexpr (BITS == 4) {
+          lraw_next[0] = __ldg(reinterpret_cast<const uint4*>(lp));
+          lraw_next[1] = __ldg(reinterpret_cast<const uint4*>(lp) + 1);
+        } else if constexpr (BITS == 3) {
+          lraw_next[0] = __ldg(reinterpret_cast<const uint4*>(lp));
+        } else {
+          const uint2 v = __ldg(reinterpret_cast<const uint2*>(lp));
+          lraw_next[0] = make_uint4(v.x, v.y, 0u, 0u);
+        }
+      }
+    };
+    fetch(0);
+    for (int i = 0; i < nsteps; ++i) {
+      const int s = i % S;
+      const Chunk<BITS> ch = ch_next;
+      const uint4 l0 = lraw_next[0], l1 = lraw_next[1];
+      const bool ok = col_ok && (int64_t)i * KS + lr < a.n;
+      if (i + 1 < nsteps) fetch(i + 1);
+      uint32_t o[16];
+      if (ok) {
+        LutRegs<BITS> L;
+        if constexpr (BITS == 4) {
+          uint32_t w[8] = {h2_to_bf2(l0.x), h2_to_bf2(l0.y), h2_to_bf2(l0.z), h2_to_bf2(l0.w),
+                           h2_to_bf2(l1.x), h2_to_bf2(l1.y), h2_to_bf2(l1.z), h2_to_bf2(l1.w)};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            L.lo[q] = prmt(w[2 * q], w[2 * q + 1], 0x6420);
+            L.hi[q] = prmt(w[2 * q], w[2 * q + 1], 0x7531);
+          }
+        } else if constexpr (BITS == 3) {
+          uint32_t w[4] = {h2_to_bf2(l0.x), h2_to_bf2(l0.y), h2_to_bf2(l0.z), h2_to_bf2(l0.w)};
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            L.lo[q] = prmt(w[2 * q], w[2 * q + 1], 0x6420);
+            L.hi[q] = prmt(w[2 * q], w[2 * q + 1], 0x7531);
+          }
+        } else {
+          const uint32_t w0 = h2_to_bf2(l0.x), w1 = h2_to_bf2(l0.y);
+          L.lo[0] = prmt(w0, w1, 0x6420);
+          L.hi[0] = prmt(w0, w1, 0x7531);
+        }
+        dequant_chunk<BITS>(ch, L, o);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) o[e] = 0u;
+      }
+      if (*abort_flag || !tc::mbar_wait(&empty[s], ((i / S) & 1) ^ 1, a.check)) { *abort_flag = 1; break; }
+      uint8_t* at = smem + s * STAGE + B_BYTES;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4*>(at + slot_off[q]) = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+      tc::fence_async_smem();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&full_a[s]);
+    }
+  }
+
+  // epilogue: thread = column j (TMEM lane), warps w and w + 4 split the tokens
+  __syncthreads();
+  if (warp < 8) {
+    const int quad = warp & 3;
+    const int64_t j = j0 + quad * 32 + lane;
+    bool have = !*abort_flag && tc::mbar_wait(d_full, 0, a.check);
+    have = __all_sync(0xffffffffu, have);  // tcgen05.ld is warp-collective
+    if (have) {
+      tc::tc_fence_after();
+      for (int gi = (warp >> 2); gi < N / 16; gi += 2) {
+        uint32_t v[16];
+        tc::tmem_ld16(tc::tmem_addr(tmem, quad * 32, gi * 16), v);
+        tc::tmem_ld_wait();
+        if (j < a.d) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int64_t t = t0 + gi * 16 + e;
+            if (t < a.T) {
+              __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(v[e]));
+              a.dX[t * a.d + j] = *reinterpret_cast<uint16_t*>(&b);
+            }
+          }
+        }
+      }
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// ============================================================================
+// dlut
+// ============================================================================
+
+namespace dl {
+constexpr int M = 128, N = 256;
+constexpr int KS = 64;          // tokens per pipeline step
+constexpr int S = 4;
+constexpr int A_BYTES = 2 * 8192;   // dY^T: two 64-row MN atoms x 8 K-groups
+constexpr int B_BYTES = 4 * 8192;   // X: four 64-column MN atoms x 8 K-groups
+constexpr int STAGE = A_BYTES + B_BYTES;
+constexpr int BAR_OFF = S * STAGE;
+constexpr int SMEM = 1024 + BAR_OFF + 256;
+constexpr int THREADS = 192;        // warps 0-3 epilogue, 4 TMA, 5 MMA
+constexpr int TMA_WARP = 4, MMA_WARP = 5;
+constexpr uint32_t IDESC = tc::idesc_bf16(M, N, 1, 1);
+constexpr int TMEM_COLS = 256;
+}  // namespace dl
+
+// Group slots of one 256-column tile: groups [tile*256 / gs, (tile*256 + 255) / gs].
+__host__ __device__ inline int dlut_slots(int64_t gs, int gpr) {
+  const int64_t s = 255 / gs + 2;
+  return (int)(s < gpr ? s : gpr);
+}
+
+struct DlutArgs {
+  const uint8_t* packed;
+  int64_t row_bytes;
+  int64_t n, d, gs, T;
+  int gpr, slots;
+  float* part;          // [jtiles][n][slots][k] partial bins
+  unsigned int* check;
+};
+
+template <int BITS>
+__global__ void __launch_bounds__(dl::THREADS, 1)
+dlut_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_x, DlutArgs a) {
+  using namespace dl;
+  constexpr int K = 1 << BITS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
+  uint64_t* empty = full + S;
+  uint64_t* d_full = empty + S;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(d_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = tc::warp_id(), lane = tc::lane_id();
+  const int jt = blockIdx.x;
+  const int64_t j0 = (int64_t)jt * N;
+  const int64_t i0 = (int64_t)blockIdx.y * M;
+  const int nsteps = ceil_div(a.T, KS);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    tc::mbar_init(d_full, 1);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == MMA_WARP) tc::tmem_alloc(tmem_slot, TMEM_COLS);
+  if (warp == TMA_WARP && lane == 0) {
+    tc::tma_prefetch(&tm_dy);
+    tc::tma_prefetch(&tm_x);
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == TMA_WARP) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < nsteps && !*abort_flag; ++i) {
+        const int s = i % S;
+        if (!tc::mbar_wait(&empty[s], ((i / S) & 1) ^ 1, a.check)) { *abort_flag = 1; break; }
+        uint8_t* st = smem + s * STAGE;
+        tc::mbar_arrive_expect_tx(&full[s], STAGE);
+        const int tk = i * KS;
+        tc::tma_load_2d(st, &tm_dy, &full[s], (int)i0, tk);
+        tc::tma_load_2d(st + 8192, &tm_dy, &full[s], (int)i0 + 64, tk);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tc::tma_load_2d(st + A_BYTES + q * 8192, &tm_x, &full[s], (int)j0 + 64 * q, tk);
+        ++issued;
+      }
+      for (int j = issued > S ? issued - S : 0; j < issued; ++j) tc::mbar_wait(&full[j % S], (j / S) & 1, a.check);
+    }
+  } else if (warp == MMA_WARP) {
+    if (lane == 0) {
+      bool ok = true;
+      for (int i = 0; i < nsteps; ++i) {
+        const int s = i % S;
+        if (*abort_flag || !tc::mbar_wait(&full[s], (i / S) & 1, a.check)) { *abort_flag = 1; ok = false; break; }
+        tc::tc_fence_after();
+        const uint32_t ab = tc::smem_u32(smem + s * STAGE), bb = ab + A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < KS / 16; ++kk) {
+          const uint64_t ad = tc::sdesc(ab + kk * 2048, 8192, 1024, tc::kSwizzle128);
+          const uint64_t bd = tc::sdesc(bb + kk * 2048, 8192, 1024, tc::kSwizzle128);
+          tc::mma_ss(tmem, ad, bd, IDESC, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc::mma_commit(&empty[s]);
+      }
+      if (ok) tc::mma_commit(d_full);
+    }
+  } else {
+    // epilogue warps 0-3: thread = row i (TMEM lane); bin the row's 256 columns
+    float* bins = reinterpret_cast<float*>(smem + BAR_OFF - K * 128 * 4);  // [K][128], tail of stage memory
+    const int tid = threadIdx.x;                                         // 0..127
+    const int64_t i = i0 + tid;
+    bool have = !*abort_flag && tc::mbar_wait(d_full, 0, a.check);
+    have = __all_sync(0xffffffffu, have);  // tcgen05.ld is warp-collective
+    if (have) tc::tc_fence_after();
+    // the bins reuse the last stage's memory: wait until every MMA has read it (d_full)
+#pragma unroll
+    for (int c = 0; c < K; ++c) bins[c * 128 + tid] = 0.f;
+    const int first_g = (int)(j0 / a.gs);
+    const int gs32 = (int)a.gs;
+    int g = first_g, g_end = (first_g + 1) * gs32;
+    bool dirty = false;
+    auto flush = [&](int gg) {
+      if (i < a.n) {
+        float* dst = a.part + (((int64_t)jt * a.n + i) * a.slots + (gg - first_g)) * K;
+#pragma unroll
+        for (int c = 0; c < K; ++c) dst[c] = bins[c * 128 + tid];
+      }
+#pragma unroll
+      for (int c = 0; c < K; ++c) bins[c * 128 + tid] = 0.f;
+    };
+    for (int q = 0; q < N / 32; ++q) {
+      const int64_t jc = j0 + 32 * q;
+      if (jc >= a.d) break;
+      uint32_t v[32];
+      if (have) {
+        tc::tmem_ld32(tc::tmem_addr(tmem, warp * 32, 32 * q), v);
+        tc::tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = 0u;
+      }
+      if ((int)jc >= g_end) {       // chunk in a later group: hand the finished group's sums on
+        if (dirty) flush(g);
+        do { ++g; g_end += gs32; } while ((int)jc >= g_end);
+        dirty = false;
+      }
+      if (i < a.n) {
+        const Chunk<BITS> ch = load_chunk<BITS>(a.packed + i * a.row_bytes, jc >> 5);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) bins[chunk_index<BITS>(ch, e) * 128 + tid] += __uint_as_float(v[e]);
+      }
+      dirty = true;
+    }
+    if (dirty) flush(g);
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == MMA_WARP) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// Sum the partial bins of every (row, group) over the column tiles that touch
+// the group, in tile order, and write (or add to) dlut.
+template <int BITS>
+__global__ void dlut_reduce_kernel(const float* __restrict__ part, int64_t n, int gpr, int64_t gs, int jtiles,
+                                   int slots, float* __restrict__ dlut, int accumulate) {
+  constexpr int K = 1 << BITS;
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= n * gpr * K) return;
+  const int c = (int)(e % K);
+  const int64_t ig = e / K;
+  const int g = (int)(ig % gpr);
+  const int64_t i = ig / gpr;
+  const int t_first = (int)(((int64_t)g * gs) / dl::N);
+  int t_last = (int)(((int64_t)(g + 1) * gs - 1) / dl::N);
+  if (t_last > jtiles - 1) t_last = jtiles - 1;
+  float sum = 0.f;
+  for (int t = t_first; t <= t_last; ++t) {
+    const int fg = (int)(((int64_t)t * dl::N) / gs);
+    sum += part[(((int64_t)t * n + i) * slots + (g - fg)) * K + c];
+  }
+  dlut[e] = accumulate ? dlut[e] + sum : sum;
+}
+
+}  // namespace
+
+size_t dlut_tc_workspace(int64_t n, int64_t d, int bits, int gpr) {
+  const int64_t gs = d / gpr;
+  const int64_t jtiles = (d + dl::N - 1) / dl::N;
+  return (size_t)jtiles * n * dlut_slots(gs, gpr) * (1 << bits) * sizeof(float);
+}
+
+cudaError_t launch_dx_tc(const Problem& p, const uint16_t* dY, uint16_t* dX, cudaStream_t s) {
+  CUtensorMap tm;
+  cudaError_t e = make_tmap_2d(&tm, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)p.n, (uint64_t)p.T,
+                               (uint64_t)p.n * 2, 64, dx::N, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
+  DxArgs args{p.packed, p.row_bytes, p.lut, p.n, p.d, p.gs, p.T, p.gpr, dX, p.check};
+  dim3 grid((unsigned)ceil_div(p.d, 128), (unsigned)ceil_div(p.T, dx::N));
+  auto run = [&](auto kern) {
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dx::SMEM);
+    if (err != cudaSuccess) return err;
+    kern<<<grid, kThreads, dx::SMEM, s>>>(tm, args);
+    return cudaGetLastError();
+  };
+  switch (p.bits) {
+    case 2: return run(dx_tc_kernel<2>);
+    case 3: return run(dx_tc_kernel<3>);
+    default: return run(dx_tc_kernel<4>);
+  }
+}
+
+cudaError_t launch_dlut_tc(const Problem& p, const uint16_t* X, const uint16_t* dY, float* dlut, int accumulate,
+                           void* workspace, cudaStream_t s) {
+  CUtensorMap tm_dy, tm_x;
+  cudaError_t e = make_tmap_2d(&tm_dy, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)p.n, (uint64_t)p.T,
+                               (uint64_t)p.n * 2, 64, dl::KS, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_2d(&tm_x, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)p.d, (uint64_t)p.T, (uint64_t)p.d * 2,
+                   64, dl::KS, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
+  const int slots = dlut_slots(p.gs, p.gpr);
+  const int jtiles = ceil_div(p.d, dl::N);
+  DlutArgs args{p.packed, p.row_bytes, p.n, p.d, p.gs, p.T, p.gpr, slots, static_cast<float*>(workspace), p.check};
+  dim3 grid((unsigned)jtiles, (unsigned)ceil_div(p.n, dl::M));
+  const int64_t outs = p.n * p.gpr * (1 << p.bits);
+  const unsigned rgrid = (unsigned)((outs + 255) / 256);
+  auto run = [&](auto kern, auto red) {
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dl::SMEM);
+    if (err != cudaSuccess) return err;
+    kern<<<grid, dl::THREADS, dl::SMEM, s>>>(tm_dy, tm_x, args);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    red<<<rgrid, 256, 0, s>>>(static_cast<const float*>(workspace), p.n, p.gpr, p.gs, jtiles, slots, dlut, accumulate);
+    return cudaGetLastError();
+  };
+  switch (p.bits) {
+    case 2: return run(dlut_tc_kernel<2>, dlut_reduce_kernel<2>);
+    case 3: return run(dlut_tc_kernel<3>, dlut_reduce_kernel<3>);
+    default: return run(dlut_tc_kernel<4>, dlut_reduce_kernel<4>);
+  }
+}
+
+}  // namespace sk

@@ -248,7 +248,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
   cg::cluster_group cluster = cg::this_cluster();
   // the accumulator is final once d_full fires; the tensor cores have then also
   // finished reading this CTA's stage memory, which becomes the split-K inbox
-  const bool have = warp < kDequantWarps && !aborted && tc::mbar_wait(d_full, 0, a.check);
+  bool have = warp < kDequantWarps && !aborted && tc::mbar_wait(d_full, 0, a.check);
+  have = __all_sync(0xffffffffu, have);  // tcgen05.ld is warp-collective
   if (have) tc::tc_fence_after();
   if (ksplit > 1) cluster.sync();  // every peer's stage memory is free now
   if (warp < kDequantWarps) {

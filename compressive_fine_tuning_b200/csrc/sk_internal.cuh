@@ -277,6 +277,10 @@ cudaError_t launch_unpack(const uint8_t* packed, int64_t n, int64_t d, int bits,
 cudaError_t launch_dequant(const Problem& p, int task, uint16_t* theta, cudaStream_t s);
 cudaError_t launch_gemv_fwd(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStream_t s);
 cudaError_t launch_fwd_tc(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStream_t s);
+cudaError_t launch_dx_tc(const Problem& p, const uint16_t* dY, uint16_t* dX, cudaStream_t s);
+cudaError_t launch_dlut_tc(const Problem& p, const uint16_t* X, const uint16_t* dY, float* dlut, int accumulate,
+                           void* workspace, cudaStream_t s);
+size_t dlut_tc_workspace(int64_t n, int64_t d, int bits, int gpr);
 cudaError_t launch_simt_bwd_input(const Problem& p, const uint16_t* dY, uint16_t* dX, cudaStream_t s);
 cudaError_t launch_simt_bwd_lut(const Problem& p, const uint16_t* X, const uint16_t* dY, float* dlut,
                                 int accumulate, cudaStream_t s);

@@ -301,3 +301,37 @@ def test_identity_exact_tc_path(fwd_path, T):
     X = torch.from_numpy(synth.make_bf16(rng, (T, n), 1.0).view(np.int16)).cuda().view(torch.bfloat16)
     Y = sk.linear_fwd(packed, lut, 2, X)
     assert torch.equal(Y.view(torch.int16), X.view(torch.int16))
+
+
+# ---------------------------------------------------------------------------
+# both backward kernels (SK_BWD_PATH forces one of them)
+# ---------------------------------------------------------------------------
+
+BWD_SHAPES = [(256, 512, 4, 1), (136, 320, 2, 5), (264, 1376, 3, 1), (128, 2752, 4, 2), (64, 512, 4, 16),
+              (1024, 4096, 2, 8)]
+
+
+@pytest.mark.parametrize("path", ["tc", "simt"])
+@pytest.mark.parametrize("shape", BWD_SHAPES)
+@pytest.mark.parametrize("T", [1, 64, 200, 513])
+def test_backward_each_path(monkeypatch, path, shape, T):
+    sk = _sk()
+    monkeypatch.setenv("SK_BWD_PATH", path)
+    c = _case(shape, T, 9500 + T)
+    packed, lut, X, dY, task = gc.dev_case(c)
+    gc.check_bwd_input(c, sk.linear_bwd_input(packed, lut, c.bits, c.d, dY, task))
+    dl = sk.linear_bwd_lut(packed, c.bits, c.gpr, X, dY, task, 1)
+    gc.check_dlut(dl.cpu().numpy()[0], oracle.backward_lut(c.x, c.dy, c.idx, c.gpr, c.k))
+    assert sk.device_check() == 0
+
+
+def test_bwd_lut_tc_workspace_required():
+    sk = _sk()
+    c = _case((256, 512, 4, 1), 128, 9600)
+    packed, lut, X, dY, task = gc.dev_case(c)
+    nb = sk.workspace_bytes(sk.SK_OP_BWD_LUT, c.n, c.d, c.bits, c.gpr, c.T, 1)
+    assert nb > 0
+    out = torch.empty((1, c.n, 1, 16), dtype=torch.float32, device="cuda")
+    st = sk.lib.sk_linear_bwd_lut(sk._ptr(packed), c.bits, c.gpr, c.n, c.d, sk._ptr(X), sk._ptr(dY), c.T, None, 1,
+                                  sk._ptr(out), 0, None, 0, None)
+    assert st == 1  # SK_ERR_INVALID_ARG: the tensor-core path needs its workspace
