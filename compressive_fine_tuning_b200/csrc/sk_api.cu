@@ -340,6 +340,49 @@ sk_status sk_linear_bwd_lut(const void* packed, int bits, int gpr, int64_t n, in
   return e == cudaSuccess ? ok() : cuda_fail(e, "LUT-gradient kernel launch");
 }
 
+sk_status sk_linear_bwd_lut_noalloc(const void* packed, int bits, int gpr, int64_t n, int64_t d, const uint16_t* X,
+                                    const uint16_t* dY, int64_t T, const int32_t* task, int ntask, float* dlut,
+                                    int accumulate, sk_stream_t stream) {
+  g_last_error.clear();
+  sk_status st = check_shape(bits, gpr, n, d, T, ntask);
+  if (st != SK_OK) return st;
+  if (accumulate != 0 && accumulate != 1) return fail(SK_ERR_INVALID_ARG, "accumulate must be 0 or 1");
+  const size_t dlut_bytes = (size_t)ntask * n * gpr * (1u << bits) * 4;
+  if (!dlut) return fail(SK_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(dlut)) return fail(SK_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (T == 0) {
+    if (accumulate) return ok();
+    cudaError_t e = cudaMemsetAsync(dlut, 0, dlut_bytes, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ok() : cuda_fail(e, "cudaMemsetAsync(dlut)");
+  }
+  st = check_layer_buffers(packed, nullptr, false, bits, gpr, n, d, T, task, ntask, X, (size_t)(T * d * 2), dY,
+                           (size_t)(T * n * 2), dlut, dlut_bytes);
+  if (st != SK_OK) return st;
+  const bool tc = use_tensor_cores_bwd(n, d, T, ntask);
+  if (tc) {
+    const size_t need = sk::dlut_tc_workspace(n, d, bits, gpr);
+    if (need > sk::dlut_noalloc_scratch_bytes())
+      return fail(SK_ERR_INVALID_ARG,
+                  "this layer needs %zu bytes of scratch but the allocation-free call holds %zu; "
+                  "use sk_linear_bwd_lut with a caller workspace", need, sk::dlut_noalloc_scratch_bytes());
+  }
+  unsigned int* check = nullptr;
+  st = device_state(&check);
+  if (st != SK_OK) return st;
+  sk::Problem p = make_problem(packed, nullptr, bits, gpr, n, d, T, task, ntask, check);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (tc) {
+    void* scratch = nullptr;
+    e = sk::dlut_noalloc_scratch(&scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "looking up the scratch array's device address");
+    e = sk::launch_dlut_tc(p, X, dY, dlut, accumulate, scratch, s);
+  } else {
+    e = sk::launch_simt_bwd_lut(p, X, dY, dlut, accumulate, s);
+  }
+  return e == cudaSuccess ? ok() : cuda_fail(e, "LUT-gradient kernel launch");
+}
+
 sk_status sk_device_check(uint32_t* flags, int clear, sk_stream_t stream) {
   g_last_error.clear();
   if (!flags) return fail(SK_ERR_INVALID_ARG, "null pointer");

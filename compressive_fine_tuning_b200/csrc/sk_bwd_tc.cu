@@ -491,3 +491,52 @@ cudaError_t launch_dlut_tc(const Problem& p, const uint16_t* X, const uint16_t* 
 }
 
 }  // namespace sk
+
+// ============================================================================
+// Allocation-free LUT gradient: the same kernels with a fixed scratch array
+// ============================================================================
+//
+// Some callers cannot allocate device memory at the point where they need the
+// LUT gradient: a plugin running inside another framework's executor that owns
+// every device allocation, a serving or training loop that has reserved all of
+// its memory up front and treats any new allocation as an error, or code that
+// must not call cudaMalloc because it synchronises the device.  For them the
+// partial bins live in one file-scope device array instead of a caller
+// workspace.  The array is reserved on every GPU that loads this library and is
+// held until the process exits.
+#include <mutex>
+
+namespace sk {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+}  // namespace
+
+size_t dlut_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+// Device address of the scratch array on the current device.  In host code the
+// array's name only stands for the host-side shadow symbol, so the device
+// address is looked up once per device (with that device current) and cached.
+cudaError_t dlut_noalloc_scratch(void** ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev] = p;
+  }
+  *ptr = g_noalloc_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace sk

@@ -281,6 +281,8 @@ cudaError_t launch_dx_tc(const Problem& p, const uint16_t* dY, uint16_t* dX, cud
 cudaError_t launch_dlut_tc(const Problem& p, const uint16_t* X, const uint16_t* dY, float* dlut, int accumulate,
                            void* workspace, cudaStream_t s);
 size_t dlut_tc_workspace(int64_t n, int64_t d, int bits, int gpr);
+size_t dlut_noalloc_scratch_bytes();
+cudaError_t dlut_noalloc_scratch(void** ptr);
 cudaError_t launch_simt_bwd_input(const Problem& p, const uint16_t* dY, uint16_t* dX, cudaStream_t s);
 cudaError_t launch_simt_bwd_lut(const Problem& p, const uint16_t* X, const uint16_t* dY, float* dlut,
                                 int accumulate, cudaStream_t s);

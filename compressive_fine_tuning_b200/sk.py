@@ -23,7 +23,7 @@ SK_CHECK_INDEX_RANGE = 2
 EXPORTED = (
     "sk_abi_version", "sk_status_string", "sk_last_error", "sk_packed_row_bytes", "sk_packed_bytes",
     "sk_pack", "sk_unpack", "sk_dequant", "sk_workspace_bytes", "sk_linear_fwd", "sk_linear_bwd_input",
-    "sk_linear_bwd_lut", "sk_device_check",
+    "sk_linear_bwd_lut", "sk_linear_bwd_lut_noalloc", "sk_device_check",
 )
 
 
@@ -51,6 +51,7 @@ def _load() -> ctypes.CDLL:
         "sk_linear_fwd": ([vp, vp, i32, i32, i64, i64, vp, i64, vp, i32, vp, vp, sz, vp], i32),
         "sk_linear_bwd_input": ([vp, vp, i32, i32, i64, i64, vp, i64, vp, i32, vp, vp, sz, vp], i32),
         "sk_linear_bwd_lut": ([vp, i32, i32, i64, i64, vp, vp, i64, vp, i32, vp, i32, vp, sz, vp], i32),
+        "sk_linear_bwd_lut_noalloc": ([vp, i32, i32, i64, i64, vp, vp, i64, vp, i32, vp, i32, vp], i32),
         "sk_device_check": ([ctypes.POINTER(ctypes.c_uint32), i32, vp], i32),
     }
     for name, (args, res) in sigs.items():

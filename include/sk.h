@@ -167,6 +167,35 @@ sk_status sk_linear_bwd_lut(const void* packed, int bits, int gpr, int64_t n, in
                             void* workspace, size_t workspace_bytes, sk_stream_t stream);
 
 /*
+ * sk_linear_bwd_lut_noalloc: the LUT gradient of sk_linear_bwd_lut, for
+ * callers that cannot allocate device memory when they need it (a plugin
+ * inside another framework's executor that owns all device memory, a loop that
+ * has reserved its whole memory budget up front, code that must not call
+ * cudaMalloc because it synchronises the device).  The pages have no
+ * counterpart: this is a deployment convenience of this library.
+ *
+ * It allocates nothing: where sk_linear_bwd_lut would take a caller workspace,
+ * this call uses one fixed array of SK_NOALLOC_SCRATCH_BYTES in device memory,
+ * reserved on every GPU that loads the library until the process exits.  The
+ * caller still passes the inputs and dlut.  Arguments, layouts, results and
+ * errors are those of sk_linear_bwd_lut; in addition a layer whose scratch
+ * need (sk_workspace_bytes(SK_OP_BWD_LUT, ...)) exceeds the array is rejected
+ * with SK_ERR_INVALID_ARG before anything is launched.
+ *
+ * The first call on a device looks up the array's device address with that
+ * device current; make that first call before any stream capture.  Every call
+ * shares the one array and it keeps the last call's contents (each call
+ * overwrites every entry it reads, so nothing has to start at zero): calls that
+ * overlap on the GPU (different streams, concurrently replayed graphs) race and
+ * corrupt each other's results, so order them on one stream.
+ */
+#define SK_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+sk_status sk_linear_bwd_lut_noalloc(const void* packed, int bits, int gpr, int64_t n, int64_t d,
+                                    const uint16_t* X, const uint16_t* dY, int64_t T,
+                                    const int32_t* task, int ntask, float* dlut, int accumulate,
+                                    sk_stream_t stream);
+
+/*
  * sk_device_check: synchronises `stream`, stores the device check word
  * (SK_CHECK_* bits, 0 = nothing flagged) in *flags and clears it if `clear`.
  * Returns SK_ERR_DEVICE_CHECK when any bit was set, else SK_OK.
