@@ -30,74 +30,84 @@ namespace cg = cooperative_groups;
 namespace sk {
 namespace {
 
-constexpr int kDequantWarps = 8;
-constexpr int kTmaWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kThreads = 320;
-constexpr int KSTEP = 128;      // weight columns per pipeline step
-constexpr int A_COLS = KSTEP / 2;  // 32-bit TMEM columns per A stage (bf16 pairs)
 
 __host__ __device__ constexpr int align1k(int x) { return (x + 1023) / 1024 * 1024; }
 __host__ __device__ constexpr int pow2ceil(int x) { int p = 32; while (p < x) p *= 2; return p; }
 
 template <int BITS, int N>
 struct Cfg {
-  // decode tiles (N <= 64) keep under half of an SM's shared and tensor memory
-  // so that the next launch's CTA can share the SM (programmatic dependent launch)
-  static constexpr int S = N >= 256 ? 3 : N >= 128 ? 5 : N >= 64 ? 4 : N >= 32 ? 6 : 8;  // shared-memory stages
-  static constexpr int SA = N <= 64 ? 3 : 2;                   // tensor-memory stages of operand A
-  static constexpr int KB = KSTEP * BITS / 8;                  // index bytes per row per step
-  static constexpr int X_BOX = N * 128;                        // one 64-column box of X
-  static constexpr int X_BYTES = 2 * X_BOX;
+  // Decode tiles (N <= 64) carry little MMA work per weight element, so the
+  // MMA -> commit -> barrier round trip (about 1.5k cycles) must be hidden by
+  // running the dequantisation many steps ahead: one CTA per SM owns all 512
+  // TMEM columns (7 A stages) and 16 dequantisation warps.  Prefill tiles are
+  // MMA-bound and keep 8 warps, 2 A stages and their deeper shared-memory ring.
+  static constexpr bool DECODE = N <= 64;
+  static constexpr int KSTEP = DECODE ? 256 : 128;            // weight columns per pipeline step
+  static constexpr int A_COLS = KSTEP / 2;                    // 32-bit TMEM columns per A stage (bf16 pairs)
+  static constexpr int DQW = DECODE ? 16 : 8;                 // dequantisation warps
+  static constexpr int TMA_WARP = DQW, MMA_WARP = DQW + 1;
+  static constexpr int THREADS = (DQW + 2) * 32;
+  static constexpr int CH = KSTEP / 32 / (DQW / 4);           // 32-column chunks per thread per step
+  static constexpr int S = N >= 256 ? 3 : N >= 128 ? 5 : N >= 64 ? 4 : N >= 32 ? 5 : 6;  // shared-memory stages
+  static constexpr int SA = DECODE ? 3 : 2;                   // tensor-memory stages of operand A
+  static constexpr int XBOXES = KSTEP / 64;                   // 64-column X boxes per step
+  static constexpr int KB = KSTEP * BITS / 8;                 // index bytes per row per step
+  static constexpr int X_BOX = N * 128;                       // one 64-column box of X
+  static constexpr int X_BYTES = XBOXES * X_BOX;
   static constexpr int IDX_OFF = align1k(X_BYTES);
   static constexpr int IDX_BYTES = 128 * KB;
   static constexpr int STAGE = IDX_OFF + align1k(IDX_BYTES);
   static constexpr int BAR_OFF = S * STAGE;
-  static constexpr int SMEM = 1024 + BAR_OFF + 256;            // + alignment slack + barriers
+  static constexpr int SMEM = 1024 + BAR_OFF + 512;           // + alignment slack + barriers
   static constexpr int D_COL = SA * A_COLS;
-  static constexpr int ROWS_PER_RANK_MAX = 128;
-  static constexpr int TMEM_COLS = pow2ceil(D_COL + N);
+  static constexpr int TMEM_COLS = 512;
   static constexpr uint32_t IDESC = tc::idesc_bf16(128, N, 0, 0);
   static_assert(N % 16 == 0 && N >= 16 && N <= 256, "UMMA N for M = 128");
-  static_assert(N * 128 * 4 <= BAR_OFF, "split-K partials reuse the stage memory");
-  static_assert(SA * A_COLS + N <= TMEM_COLS, "tensor memory budget");
+  static_assert(N * (128 + 8) * 4 <= BAR_OFF, "split-K partials reuse the stage memory");
+  static_assert(D_COL + N <= TMEM_COLS, "tensor memory budget");
+  static_assert(SMEM <= 232448, "shared memory budget");
 };
 
 struct FwdArgs {
   const uint16_t* lut;
   int64_t n, d, gs, T;
   int gpr;
-  int steps_total;  // ceil(d / KSTEP)
+  int steps_total;  // ceil(d / C::KSTEP)
   uint16_t* Y;
   unsigned int* check;
 };
 
-// The thread's two 32-column chunks of the step (half h of the 128 columns),
-// read from the TMA-swizzled index tile.
-template <int BITS>
-__device__ __forceinline__ void read_idx(const uint8_t* tile, int r, int h, Chunk<BITS> (&ch)[2]) {
-  if constexpr (BITS == 4) {         // 64-byte rows, 64B swizzle: chunk q at q ^ ((r >> 1) & 3)
-    const int sw = (r >> 1) & 3;
+// The thread's CH consecutive 32-column chunks of the step, starting at chunk
+// c0, read from the TMA-swizzled index tile whose rows are KB bytes (the TMA
+// swizzle span equals KB when KB is 32, 64 or 128 bytes: the 16-byte piece p
+// of row r sits at p ^ ((r * KB / 128) % (KB / 16))).
+template <int BITS, int KB, int CH>
+__device__ __forceinline__ void read_idx(const uint8_t* tile, int r, int c0, Chunk<BITS> (&ch)[CH]) {
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const uint4 v = *reinterpret_cast<const uint4*>(tile + r * 64 + 16 * ((2 * h + c) ^ sw));
-      ch[c].w[0] = v.x; ch[c].w[1] = v.y; ch[c].w[2] = v.z; ch[c].w[3] = v.w;
+  for (int c = 0; c < CH; ++c) {
+    const int q = c0 + c;
+    if constexpr (BITS == 4 || BITS == 2) {
+      constexpr int PIECES = KB / 16;                       // 16-byte pieces per row
+      const int sw = ((r * KB) >> 7) & (PIECES - 1);
+      if constexpr (BITS == 4) {                            // one chunk per piece
+        const uint4 v = *reinterpret_cast<const uint4*>(tile + r * KB + 16 * (q ^ sw));
+        ch[c].w[0] = v.x; ch[c].w[1] = v.y; ch[c].w[2] = v.z; ch[c].w[3] = v.w;
+      } else {                                              // two chunks per piece
+        const uint2 v = *reinterpret_cast<const uint2*>(tile + r * KB + 16 * ((q >> 1) ^ sw) + 8 * (q & 1));
+        ch[c].w[0] = v.x; ch[c].w[1] = v.y;
+      }
+    } else {                                                // 3-bit: unswizzled rows, 12 bytes per chunk
+      const uint32_t* p = reinterpret_cast<const uint32_t*>(tile + r * KB + 12 * q);
+      ch[c].w[0] = p[0]; ch[c].w[1] = p[1]; ch[c].w[2] = p[2];
     }
-  } else if constexpr (BITS == 2) {  // 32-byte rows, 32B swizzle: chunk q at q ^ ((r >> 2) & 1)
-    const uint4 v = *reinterpret_cast<const uint4*>(tile + r * 32 + 16 * (h ^ ((r >> 2) & 1)));
-    ch[0].w[0] = v.x; ch[0].w[1] = v.y; ch[1].w[0] = v.z; ch[1].w[1] = v.w;
-  } else {                           // 48-byte rows, no swizzle (conflict-free as is)
-    const uint2* p = reinterpret_cast<const uint2*>(tile + r * 48 + 24 * h);
-    const uint2 a = p[0], b = p[1], c = p[2];
-    ch[0].w[0] = a.x; ch[0].w[1] = a.y; ch[0].w[2] = b.x;
-    ch[1].w[0] = b.y; ch[1].w[1] = c.x; ch[1].w[2] = c.y;
   }
 }
 
 template <int BITS, int N>
-__global__ void __launch_bounds__(kThreads, N <= 64 ? 2 : 1)
+__global__ void __launch_bounds__(Cfg<BITS, N>::THREADS, 1)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_idx, FwdArgs a) {
   using C = Cfg<BITS, N>;
+  constexpr int kDequantWarps = C::DQW, kTmaWarp = C::TMA_WARP, kMmaWarp = C::MMA_WARP, kThreads = C::THREADS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
@@ -153,9 +163,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         if (!tc::mbar_wait(&empty[s], ((i / C::S) & 1) ^ 1, a.check)) { *abort_flag = 1; break; }
         uint8_t* st = smem + s * C::STAGE;
         tc::mbar_arrive_expect_tx(&full[s], C::X_BYTES + C::IDX_BYTES);
-        const int k0 = (s0 + i) * KSTEP;
-        tc::tma_load_2d(st, &tm_x, &full[s], k0, t0);
-        tc::tma_load_2d(st + C::X_BOX, &tm_x, &full[s], k0 + 64, t0);
+        const int k0 = (s0 + i) * C::KSTEP;
+#pragma unroll
+        for (int b = 0; b < C::XBOXES; ++b) tc::tma_load_2d(st + b * C::X_BOX, &tm_x, &full[s], k0 + 64 * b, t0);
         tc::tma_load_2d(st + C::IDX_OFF, &tm_idx, &full[s], (s0 + i) * C::KB, (int)m0);
         ++issued;
       }
@@ -167,6 +177,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
     // ---------------- MMA issue ----------------
     if (lane == 0) {
       bool ok = true;
+      const uint64_t desc0 = tc::sdesc(tc::smem_u32(smem), 16, 1024, tc::kSwizzle128);
       for (int i = 0; i < nsteps; ++i) {
         const int s = i % C::S, ai = i % SA;
         if (*abort_flag || !tc::mbar_wait(&full[s], (i / C::S) & 1, a.check) ||
@@ -174,11 +185,14 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
           *abort_flag = 1; ok = false; break;
         }
         tc::tc_fence_after();
-        const uint32_t xb = tc::smem_u32(smem + s * C::STAGE);
+        // descriptor of this stage's X tile; the start-address field (bits 0..13,
+        // 16-byte units) absorbs the per-MMA offsets without carrying out
+        const uint64_t bd0 = desc0 + (uint64_t)((s * C::STAGE) >> 4);
+        const uint32_t a0 = tmem + ai * C::A_COLS;
 #pragma unroll
-        for (int kk = 0; kk < KSTEP / 16; ++kk) {
-          const uint64_t bd = tc::sdesc(xb + (kk >> 2) * C::X_BOX + (kk & 3) * 32, 16, 1024, tc::kSwizzle128);
-          tc::mma_ts(tmem + C::D_COL, tmem + ai * A_COLS + kk * 8, bd, C::IDESC, (i > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < C::KSTEP / 16; ++kk) {
+          const uint64_t bd = bd0 + (uint64_t)(((kk >> 2) * C::X_BOX + (kk & 3) * 32) >> 4);
+          tc::mma_ts(tmem + C::D_COL, a0 + kk * 8, bd, C::IDESC, (i > 0 || kk > 0) ? 1u : 0u);
         }
         tc::mma_commit(&empty[s]);
         tc::mma_commit(&a_empty[ai]);
@@ -187,39 +201,51 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
     }
   } else {
     // ---------------- dequantisation into tensor memory ----------------
-    const int quad = warp & 3, h = warp >> 2;
+    // warp w owns TMEM lanes 32 (w % 4) .. + 31 (its 32 rows) and chunks
+    // [part * CH, part * CH + CH) of every 128-column step
+    constexpr int CH = C::CH;
+    const int quad = warp & 3, part = warp >> 2;
     const int r = quad * 32 + lane;
     const int64_t row = m0 + r;
     const bool row_ok = row < a.n;
     const uint16_t* lut_row = a.lut + (row_ok ? row : 0) * a.gpr * (1 << BITS);
     // group bookkeeping in 32-bit arithmetic, advanced incrementally (no divisions in the loop)
     const int d32 = (int)a.d, gs32 = (int)a.gs;
-    int col = s0 * KSTEP + h * 64;          // first column of this thread's half of the step
+    int col = s0 * C::KSTEP + part * CH * 32;  // first column of this thread's chunks in the step
     int g = col / gs32;
     if (g >= a.gpr) g = a.gpr - 1;
     int g_end = (g + 1) * gs32;             // first column past group g
-    // fetch the first group's table now, overlapping the first TMA round trip
+    // fetch the first group's table now, overlapping the first TMA round trip,
+    // and always keep the next group's raw table in flight
     LutRegs<BITS> L;
+    LutRaw<BITS> nxt;
     load_lut<BITS>(lut_row + g * (1 << BITS), L);
-    for (int i = 0; i < nsteps; ++i, col += KSTEP) {
+    fetch_lut<BITS>(lut_row + (g + 1 < a.gpr ? g + 1 : g) * (1 << BITS), nxt);
+    for (int i = 0; i < nsteps; ++i, col += C::KSTEP) {
       const int s = i % C::S, ai = i % SA;
       if (*abort_flag || !tc::mbar_wait(&full[s], (i / C::S) & 1, a.check) ||
           !tc::mbar_wait(&a_empty[ai], ((i / SA) & 1) ^ 1, a.check)) {
         *abort_flag = 1; break;
       }
       tc::tc_fence_after();
-      Chunk<BITS> ch[2];
-      read_idx<BITS>(smem + s * C::STAGE + C::IDX_OFF, r, h, ch);
+      Chunk<BITS> ch[CH];
+      read_idx<BITS, C::KB, CH>(smem + s * C::STAGE + C::IDX_OFF, r, part * CH, ch);
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&empty[s]);
-      uint32_t v[32];
+      uint32_t v[16 * CH];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < CH; ++c) {
         const int cc = col + 32 * c;
         if (row_ok && cc < d32) {
           if (cc >= g_end) {             // a chunk never straddles groups (gs % 32 == 0)
-            do { ++g; g_end += gs32; } while (cc >= g_end);
-            load_lut<BITS>(lut_row + g * (1 << BITS), L);
+            ++g; g_end += gs32;
+            if (cc >= g_end) {             // skipped a whole group: fetch directly
+              do { ++g; g_end += gs32; } while (cc >= g_end);
+              load_lut<BITS>(lut_row + g * (1 << BITS), L);
+            } else {
+              to_lut<BITS>(nxt, L);
+            }
+            fetch_lut<BITS>(lut_row + (g + 1 < a.gpr ? g + 1 : g) * (1 << BITS), nxt);
           }
           uint32_t o[16];
           dequant_chunk<BITS>(ch[c], L, o);
@@ -230,7 +256,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
           for (int e = 0; e < 16; ++e) v[16 * c + e] = 0u;
         }
       }
-      tc::tmem_st32(tc::tmem_addr(tmem, quad * 32, ai * A_COLS + h * 32), v);
+      const uint32_t taddr = tc::tmem_addr(tmem, quad * 32, ai * C::A_COLS + part * CH * 16);
+      if constexpr (CH == 2) {
+        tc::tmem_st32(taddr, v);
+      } else {
+        tc::tmem_st16(taddr, v);
+      }
       tc::tmem_st_wait();
       tc::tc_fence_before();
       __syncwarp();
@@ -241,9 +272,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
   // ---------------- epilogue ----------------
   __syncthreads();
   const bool aborted = *abort_flag != 0;
-  // split-K: rows [q * rows_per, (q + 1) * rows_per) of every CTA's partial go
-  // to cluster rank q, slot = the sender's rank; layout [slot][N][rows_per]
-  const int rows_per = 128 / ksplit;
+  // split-K: cluster rank q owns rows [q * 128 / ksplit, (q + 1) * 128 / ksplit)
+  // of the tile; every CTA pushes those rows of its partial into rank q's
+  // inbox at slot = its own rank.  Inbox layout [slot][N][RP], RP = ceil(128 / ksplit).
+  const int RP = (128 + ksplit - 1) / ksplit;
   float* inbox = reinterpret_cast<float*>(smem);
   cg::cluster_group cluster = cg::this_cluster();
   // the accumulator is final once d_full fires; the tensor cores have then also
@@ -253,12 +285,16 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
   if (have) tc::tc_fence_after();
   if (ksplit > 1) cluster.sync();  // every peer's stage memory is free now
   if (warp < kDequantWarps) {
-    const int quad = warp & 3;
+    constexpr int PARTS = kDequantWarps / 4;
+    const int quad = warp & 3, part = warp >> 2;
     const int r = quad * 32 + lane;
     const int64_t row = m0 + r;
+    int q = (r * ksplit) / 128;              // owner rank of row r
+    while ((q + 1) * 128 / ksplit <= r) ++q;
+    while (q * 128 / ksplit > r) --q;
+    const int rr = r - q * 128 / ksplit;
     constexpr int GROUPS = N / 16;
-    // warps w and w + 4 share a lane quadrant and split the N columns
-    for (int gi = warp >> 2; gi < GROUPS; gi += 2) {
+    for (int gi = part; gi < GROUPS; gi += PARTS) {
       uint32_t v[16];
       if (have) {
         tc::tmem_ld16(tc::tmem_addr(tmem, quad * 32, C::D_COL + gi * 16), v);
@@ -279,20 +315,20 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
           }
         }
       } else {
-        const int q = r / rows_per, rr = r % rows_per;
-        float* dst = cluster.map_shared_rank(inbox, q) + (ks * N + gi * 16) * rows_per + rr;
+        float* dst = cluster.map_shared_rank(inbox, q) + (ks * N + gi * 16) * RP + rr;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) dst[j * rows_per] = __uint_as_float(v[j]);
+        for (int j = 0; j < 16; ++j) dst[j * RP] = __uint_as_float(v[j]);
       }
     }
   }
   if (ksplit > 1) {
     cluster.sync();  // all pushes landed
-    for (int e = threadIdx.x; e < N * rows_per; e += kThreads) {
-      const int t = e / rows_per, rr = e % rows_per;
+    const int lo = ks * 128 / ksplit, rows_mine = (ks + 1) * 128 / ksplit - lo;
+    for (int e = threadIdx.x; e < N * rows_mine; e += kThreads) {
+      const int t = e / rows_mine, rr = e % rows_mine;
       float sum = 0.f;
-      for (int q = 0; q < ksplit; ++q) sum += inbox[(q * N + t) * rows_per + rr];
-      const int64_t tg = t0 + t, row = m0 + ks * rows_per + rr;
+      for (int qq = 0; qq < ksplit; ++qq) sum += inbox[(qq * N + t) * RP + rr];
+      const int64_t tg = t0 + t, row = m0 + lo + rr;
       if (tg < a.T && row < a.n) {
         __nv_bfloat16 b = __float2bfloat16_rn(sum);
         a.Y[tg * a.n + row] = *reinterpret_cast<uint16_t*>(&b);
@@ -316,27 +352,32 @@ cudaError_t launch_n(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStrea
   e = make_tmap_2d(&tm_x, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)p.d, (uint64_t)p.T,
                                (uint64_t)p.d * 2, 64, N, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
-  const CUtensorMapSwizzle isw = BITS == 4 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                 : BITS == 2 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_NONE;
+  const CUtensorMapSwizzle isw = BITS == 3 ? CU_TENSOR_MAP_SWIZZLE_NONE
+                                 : C::KB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                 : C::KB == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
   e = make_tmap_2d(&tm_idx, p.packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)p.row_bytes, (uint64_t)p.n,
                    (uint64_t)p.row_bytes, C::KB, 128, isw);
   if (e != cudaSuccess) return e;
 
-  const int steps = (int)((p.d + KSTEP - 1) / KSTEP);
+  const int steps = (int)((p.d + C::KSTEP - 1) / C::KSTEP);
   const int64_t m_blocks = (p.n + 127) / 128;
   const int64_t t_tiles = (p.T + N - 1) / N;
   int ksplit = 1;
-  if (N <= 64) {
-    const int64_t target = 2 * (int64_t)num_sms();
-    while (ksplit < 8 && m_blocks * t_tiles * ksplit * 2 <= target && ksplit * 2 <= steps) ksplit *= 2;
+  if (C::DECODE) {
+    // the largest split (<= 8 CTAs per cluster, >= 2 steps each) that keeps the
+    // grid within one wave of one CTA per SM
+    const int64_t sms = num_sms();
+    for (int k = 8; k >= 1; --k) {
+      if (m_blocks * t_tiles * k <= sms && 2 * k <= steps) { ksplit = k; break; }
+    }
     const int forced = env_int("SK_TC_KSPLIT", 0);
-    if (forced == 1 || forced == 2 || forced == 4 || forced == 8) ksplit = forced <= steps ? forced : 1;
+    if (forced >= 1 && forced <= 8) ksplit = forced <= steps ? forced : 1;
   }
   FwdArgs args{p.lut, p.n, p.d, p.gs, p.T, p.gpr, steps, Y, p.check};
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)ksplit, (unsigned)m_blocks, (unsigned)t_tiles);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(C::THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];

@@ -122,6 +122,49 @@ __device__ __forceinline__ void load_lut(const uint16_t* __restrict__ p, LutRegs
   }
 }
 
+// Raw fp16 words of one table, fetched ahead of time; `to_lut` converts them.
+template <int BITS>
+struct LutRaw {
+  uint4 a, b;
+};
+
+template <int BITS>
+__device__ __forceinline__ void fetch_lut(const uint16_t* __restrict__ p, LutRaw<BITS>& r) {
+  if constexpr (BITS == 4) {
+    r.a = __ldg(reinterpret_cast<const uint4*>(p));
+    r.b = __ldg(reinterpret_cast<const uint4*>(p) + 1);
+  } else if constexpr (BITS == 3) {
+    r.a = __ldg(reinterpret_cast<const uint4*>(p));
+  } else {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+    r.a = make_uint4(v.x, v.y, 0u, 0u);
+  }
+}
+
+template <int BITS>
+__device__ __forceinline__ void to_lut(const LutRaw<BITS>& r, LutRegs<BITS>& L) {
+  if constexpr (BITS == 4) {
+    uint32_t w[8] = {h2_to_bf2(r.a.x), h2_to_bf2(r.a.y), h2_to_bf2(r.a.z), h2_to_bf2(r.a.w),
+                     h2_to_bf2(r.b.x), h2_to_bf2(r.b.y), h2_to_bf2(r.b.z), h2_to_bf2(r.b.w)};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      L.lo[q] = prmt(w[2 * q], w[2 * q + 1], 0x6420);
+      L.hi[q] = prmt(w[2 * q], w[2 * q + 1], 0x7531);
+    }
+  } else if constexpr (BITS == 3) {
+    uint32_t w[4] = {h2_to_bf2(r.a.x), h2_to_bf2(r.a.y), h2_to_bf2(r.a.z), h2_to_bf2(r.a.w)};
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      L.lo[q] = prmt(w[2 * q], w[2 * q + 1], 0x6420);
+      L.hi[q] = prmt(w[2 * q], w[2 * q + 1], 0x7531);
+    }
+  } else {
+    const uint32_t w0 = h2_to_bf2(r.a.x), w1 = h2_to_bf2(r.a.y);
+    L.lo[0] = prmt(w0, w1, 0x6420);
+    L.hi[0] = prmt(w0, w1, 0x7531);
+  }
+}
+
 // ----------------------------------------------------------------------------
 // packed chunks of 32 indices
 // ----------------------------------------------------------------------------
