@@ -117,6 +117,9 @@ bool use_tensor_cores_fwd(const sk::Problem& p) {
   return tc_ok && p.T >= kFwdTcMinT;
 }
 
+// Several LUT sets: the tensor-core forward needs the routing workspace.
+bool routed_fwd_possible(int64_t d, int ntask) { return ntask > 1 && ntask <= sk::kMaxRouteTasks && d >= 128; }
+
 // Shape rules shared by the layer calls.
 sk_status check_shape(int bits, int gpr, int64_t n, int64_t d, int64_t T, int ntask) {
   if (bits < 2 || bits > 4) return fail(SK_ERR_INVALID_ARG, "bits must be 2, 3 or 4 (got %d)", bits);
@@ -237,6 +240,7 @@ size_t sk_workspace_bytes(int op, int64_t n, int64_t d, int bits, int gpr, int64
   if (bits < 2 || bits > 4 || n < 1 || d < 32 || gpr < 1 || d % gpr != 0 || T < 1) return 0;
   if (op == SK_OP_BWD_LUT && use_tensor_cores_bwd(n, d, T, ntask))
     return sk::dlut_tc_workspace(n, d, bits, gpr);
+  if (op == SK_OP_FWD && routed_fwd_possible(d, ntask)) return sk::fwd_tc_workspace(T, d, ntask);
   return 0;
 }
 
@@ -268,14 +272,27 @@ sk_status sk_linear_fwd(const void* packed, const uint16_t* lut, int bits, int g
   st = check_layer_buffers(packed, lut, true, bits, gpr, n, d, T, task, ntask, X, (size_t)(T * d * 2), nullptr, 0, Y,
                            (size_t)(T * n * 2));
   if (st != SK_OK) return st;
-  if (workspace_bytes < sk_workspace_bytes(SK_OP_FWD, n, d, bits, gpr, T, ntask))
-    return fail(SK_ERR_INVALID_ARG, "workspace too small");
   unsigned int* check = nullptr;
   st = device_state(&check);
   if (st != SK_OK) return st;
   sk::Problem p = make_problem(packed, lut, bits, gpr, n, d, T, task, ntask, check);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = use_tensor_cores_fwd(p) ? sk::launch_fwd_tc(p, X, Y, s) : sk::launch_gemv_fwd(p, X, Y, s);
+  cudaError_t e;
+  if (task != nullptr && routed_fwd_possible(d, ntask)) {
+    // several LUT sets: bucket the tokens by task and run the tensor-core
+    // forward per task tile when the caller gave the routing workspace; without
+    // it (or with SK_FWD_PATH=gemv) the CUDA-core kernel serves the batch
+    const size_t need = sk::fwd_tc_workspace(T, d, ntask);
+    const bool ws_ok = workspace != nullptr && workspace_bytes >= need && aligned16(workspace) &&
+                       !overlaps(workspace, need, X, (size_t)(T * d * 2)) && !overlaps(workspace, need, Y, (size_t)(T * n * 2));
+    if (ws_ok && env_path("SK_FWD_PATH") != 1) {
+      e = sk::launch_fwd_tc_routed(p, X, Y, workspace, s);
+    } else {
+      e = sk::launch_gemv_fwd(p, X, Y, s);
+    }
+  } else {
+    e = use_tensor_cores_fwd(p) ? sk::launch_fwd_tc(p, X, Y, s) : sk::launch_gemv_fwd(p, X, Y, s);
+  }
   return e == cudaSuccess ? ok() : cuda_fail(e, "forward kernel launch");
 }
 

@@ -75,6 +75,12 @@ struct FwdArgs {
   int steps_total;  // ceil(d / C::KSTEP)
   uint16_t* Y;
   unsigned int* check;
+  // task-routed batches: X rows are in task order, tile z covers positions
+  // [tiles[3z + 1], + tiles[3z + 2]) of task tiles[3z] and perm maps a position
+  // back to its token; nullptr for single-LUT-set batches
+  const int* tiles;
+  const int* perm;
+  int64_t lut_task_stride;  // elements between consecutive LUT sets
 };
 
 // The thread's CH consecutive 32-column chunks of the step, starting at chunk
@@ -124,7 +130,22 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
   const int warp = tc::warp_id(), lane = tc::lane_id();
   const int ks = blockIdx.x, ksplit = gridDim.x;
   const int64_t m0 = (int64_t)blockIdx.y * 128;
-  const int t0 = blockIdx.z * N;
+  int t0 = blockIdx.z * N;       // first X row of the tile
+  int tlen = N;                  // tokens of the tile (bounded by T below)
+  const uint16_t* lut = a.lut;
+  if (a.tiles != nullptr) {
+    // the routing kernel wrote the tile list: wait for it before the setup
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int tau = a.tiles[3 * blockIdx.z];
+    t0 = a.tiles[3 * blockIdx.z + 1];
+    tlen = a.tiles[3 * blockIdx.z + 2];
+    if (tlen == 0) return;       // the whole cluster shares the tile and leaves together
+    lut += (int64_t)tau * a.lut_task_stride;
+  } else if (t0 + tlen > a.T) {
+    tlen = (int)(a.T - t0);
+  }
+  // output row of tile token t (positions map back to tokens when routed)
+  auto out_row = [&](int t) -> int64_t { return a.tiles != nullptr ? (int64_t)a.perm[t0 + t] : (int64_t)(t0 + t); };
   const int s0 = (int)((int64_t)ks * a.steps_total / ksplit);
   const int s1 = (int)((int64_t)(ks + 1) * a.steps_total / ksplit);
   const int nsteps = s1 - s0;
@@ -152,7 +173,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // inputs may come from the previous launch: wait for it before reading any
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (a.tiles == nullptr) asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == kTmaWarp) {
     // ---------------- producer: TMA loads ----------------
@@ -208,7 +229,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
     const int r = quad * 32 + lane;
     const int64_t row = m0 + r;
     const bool row_ok = row < a.n;
-    const uint16_t* lut_row = a.lut + (row_ok ? row : 0) * a.gpr * (1 << BITS);
+    const uint16_t* lut_row = lut + (row_ok ? row : 0) * a.gpr * (1 << BITS);
     // group bookkeeping in 32-bit arithmetic, advanced incrementally (no divisions in the loop)
     const int d32 = (int)a.d, gs32 = (int)a.gs;
     int col = s0 * C::KSTEP + part * CH * 32;  // first column of this thread's chunks in the step
@@ -307,10 +328,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         if (row < a.n) {
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const int64_t t = t0 + gi * 16 + j;
-            if (t < a.T) {
+            const int t = gi * 16 + j;
+            if (t < tlen) {
               __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(v[j]));
-              a.Y[t * a.n + row] = *reinterpret_cast<uint16_t*>(&b);
+              a.Y[out_row(t) * a.n + row] = *reinterpret_cast<uint16_t*>(&b);
             }
           }
         }
@@ -328,10 +349,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
       const int t = e / rows_mine, rr = e % rows_mine;
       float sum = 0.f;
       for (int qq = 0; qq < ksplit; ++qq) sum += inbox[(qq * N + t) * RP + rr];
-      const int64_t tg = t0 + t, row = m0 + lo + rr;
-      if (tg < a.T && row < a.n) {
+      const int64_t row = m0 + lo + rr;
+      if (t < tlen && row < a.n) {
         __nv_bfloat16 b = __float2bfloat16_rn(sum);
-        a.Y[tg * a.n + row] = *reinterpret_cast<uint16_t*>(&b);
+        a.Y[out_row(t) * a.n + row] = *reinterpret_cast<uint16_t*>(&b);
       }
     }
   }
@@ -344,12 +365,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
 }
 
 template <int BITS, int N>
-cudaError_t launch_n(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStream_t s) {
+cudaError_t launch_n(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStream_t s, const Routed* rt = nullptr) {
   using C = Cfg<BITS, N>;
   cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<BITS, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   CUtensorMap tm_x, tm_idx;
-  e = make_tmap_2d(&tm_x, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)p.d, (uint64_t)p.T,
+  e = make_tmap_2d(&tm_x, rt != nullptr ? rt->Xp : X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)p.d, (uint64_t)p.T,
                                (uint64_t)p.d * 2, 64, N, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
   const CUtensorMapSwizzle isw = BITS == 3 ? CU_TENSOR_MAP_SWIZZLE_NONE
@@ -361,7 +382,7 @@ cudaError_t launch_n(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStrea
 
   const int steps = (int)((p.d + C::KSTEP - 1) / C::KSTEP);
   const int64_t m_blocks = (p.n + 127) / 128;
-  const int64_t t_tiles = (p.T + N - 1) / N;
+  const int64_t t_tiles = rt != nullptr ? rt->max_tiles : (p.T + N - 1) / N;
   int ksplit = 1;
   if (C::DECODE) {
     // the largest split (<= 8 CTAs per cluster, >= 2 steps each) that keeps the
@@ -373,7 +394,9 @@ cudaError_t launch_n(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStrea
     const int forced = env_int("SK_TC_KSPLIT", 0);
     if (forced >= 1 && forced <= 8) ksplit = forced <= steps ? forced : 1;
   }
-  FwdArgs args{p.lut, p.n, p.d, p.gs, p.T, p.gpr, steps, Y, p.check};
+  FwdArgs args{p.lut, p.n, p.d, p.gs, p.T, p.gpr, steps, Y, p.check,
+               rt != nullptr ? rt->tiles : nullptr, rt != nullptr ? rt->perm : nullptr,
+               p.n * p.gpr * (1 << BITS)};
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)ksplit, (unsigned)m_blocks, (unsigned)t_tiles);
@@ -393,6 +416,21 @@ cudaError_t launch_n(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStrea
 }
 
 template <int BITS>
+cudaError_t launch_bits_routed(const Problem& p, const uint16_t* X, uint16_t* Y, void* ws, cudaStream_t s) {
+  const int N = fwd_tc_tile_n(p.T, p.ntask);
+  Routed rt;
+  cudaError_t e = launch_route(p, X, Y, N, ws, &rt, s);
+  if (e != cudaSuccess) return e;
+  switch (N) {
+    case 16: return launch_n<BITS, 16>(p, X, Y, s, &rt);
+    case 32: return launch_n<BITS, 32>(p, X, Y, s, &rt);
+    case 64: return launch_n<BITS, 64>(p, X, Y, s, &rt);
+    case 128: return launch_n<BITS, 128>(p, X, Y, s, &rt);
+    default: return launch_n<BITS, 256>(p, X, Y, s, &rt);
+  }
+}
+
+template <int BITS>
 cudaError_t launch_bits(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStream_t s) {
   if (p.T <= 16) return launch_n<BITS, 16>(p, X, Y, s);
   if (p.T <= 32) return launch_n<BITS, 32>(p, X, Y, s);
@@ -402,6 +440,26 @@ cudaError_t launch_bits(const Problem& p, const uint16_t* X, uint16_t* Y, cudaSt
 }
 
 }  // namespace
+
+int fwd_tc_tile_n(int64_t T, int ntask) {
+  const int64_t per = (T + ntask - 1) / ntask;   // tokens per task on average
+  return per <= 16 ? 16 : per <= 32 ? 32 : per <= 64 ? 64 : per <= 128 ? 128 : 256;
+}
+
+size_t fwd_tc_workspace(int64_t T, int64_t d, int ntask) {
+  return route_workspace_bytes(T, d, ntask, fwd_tc_tile_n(T, ntask));
+}
+
+cudaError_t launch_fwd_tc_routed(const Problem& p, const uint16_t* X, uint16_t* Y, void* ws, cudaStream_t s) {
+  cudaError_t e;
+  switch (p.bits) {
+    case 2: e = launch_bits_routed<2>(p, X, Y, ws, s); break;
+    case 3: e = launch_bits_routed<3>(p, X, Y, ws, s); break;
+    default: e = launch_bits_routed<4>(p, X, Y, ws, s); break;
+  }
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
 
 cudaError_t launch_fwd_tc(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStream_t s) {
   cudaError_t e;

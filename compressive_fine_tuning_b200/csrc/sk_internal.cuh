@@ -307,6 +307,24 @@ __device__ __forceinline__ const uint16_t* lut_ptr(const Problem& p, int tau, in
   return p.lut + (((int64_t)tau * p.n + i) * p.gpr + g) * (1 << p.bits);
 }
 
+// Task routing for the tensor-core forward (sk_route.cu).
+constexpr int kMaxRouteTasks = 256;
+struct Routed {
+  const int* perm;   // [T] position in task order -> token
+  const int* tiles;  // [max_tiles][3] (task, first position, length); length 0 = empty
+  int max_tiles;
+  const uint16_t* Xp;  // [T][d] X rows in task order
+};
+int route_max_tiles(int64_t T, int ntask, int N);
+size_t route_workspace_bytes(int64_t T, int64_t d, int ntask, int N);
+cudaError_t launch_route(const Problem& p, const uint16_t* X, uint16_t* Y, int N, void* workspace, Routed* out,
+                         cudaStream_t s);
+// Token tile of the tensor-core forward for a batch of T tokens spread over
+// ntask LUT sets (16 ... 256).
+int fwd_tc_tile_n(int64_t T, int ntask);
+size_t fwd_tc_workspace(int64_t T, int64_t d, int ntask);
+cudaError_t launch_fwd_tc_routed(const Problem& p, const uint16_t* X, uint16_t* Y, void* workspace, cudaStream_t s);
+
 // Host-side knobs read from the environment (experiments and tests).
 int env_int(const char* name, int dflt);
 // Programmatic dependent launch for the forward kernels (SK_PDL=0 turns it off).

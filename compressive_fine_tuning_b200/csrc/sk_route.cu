@@ -1,0 +1,115 @@
+// Task routing for the tensor-core forward ("SpaLLM: Unified Compressive
+// Adaptation of LLMs with Sketching", section 2.3: several LUT sets share one
+// index map; every token uses its own task's set).
+//
+// The tensor-core tiles need one LUT set per tile, so the tokens are bucketed
+// by task first:
+//   * route_kernel (one CTA) counts the tokens of every task, lays the tasks'
+//     segments out back to back, writes the permutation perm[position] = token
+//     and the tile list (task, first position, length) with at most N tokens
+//     per tile; tokens with an out-of-range task id are left out, flagged in
+//     the check word and get a zero output row;
+//   * gather_kernel copies X's rows into segment order.
+// The forward kernel then runs over the tiles and scatters each output row
+// back to its token.  A token's output does not depend on which other tokens
+// share its tile, so the order inside a segment does not matter.
+#include "sk_internal.cuh"
+
+namespace sk {
+namespace {
+
+constexpr int kRouteThreads = 1024;
+
+// workspace layout (4-byte words): perm[T] | tiles[max_tiles * 3] | valid[1], then X_perm (16-byte aligned)
+__global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __restrict__ task, int T, int ntask, int N,
+                                                              int* __restrict__ perm, int* __restrict__ tiles,
+                                                              int max_tiles, int* __restrict__ valid,
+                                                              uint16_t* __restrict__ Y, int64_t n, unsigned int* check) {
+  __shared__ int cnt[kMaxRouteTasks], off[kMaxRouteTasks + 1], cur[kMaxRouteTasks];
+  for (int i = threadIdx.x; i < ntask; i += kRouteThreads) {
+    cnt[i] = 0;
+    cur[i] = 0;
+  }
+  __syncthreads();
+  for (int t = threadIdx.x; t < T; t += kRouteThreads) {
+    const int tau = task[t];
+    if (tau >= 0 && tau < ntask) {
+      atomicAdd(&cnt[tau], 1);
+    } else {
+      atomicOr(check, SK_CHECK_TASK_RANGE);
+      for (int64_t i = 0; i < n; ++i) Y[(int64_t)t * n + i] = 0;  // rare: flagged tokens get zeros
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0, nt = 0;
+    for (int tau = 0; tau < ntask; ++tau) {
+      off[tau] = acc;
+      for (int k = 0; k < cnt[tau]; k += N) {
+        tiles[3 * nt + 0] = tau;
+        tiles[3 * nt + 1] = acc + k;
+        tiles[3 * nt + 2] = cnt[tau] - k < N ? cnt[tau] - k : N;
+        ++nt;
+      }
+      acc += cnt[tau];
+    }
+    off[ntask] = acc;
+    *valid = acc;
+    for (; nt < max_tiles; ++nt) {
+      tiles[3 * nt + 0] = 0;
+      tiles[3 * nt + 1] = 0;
+      tiles[3 * nt + 2] = 0;  // empty tile: its CTAs exit at once
+    }
+  }
+  __syncthreads();
+  for (int t = threadIdx.x; t < T; t += kRouteThreads) {
+    const int tau = task[t];
+    if (tau >= 0 && tau < ntask) perm[off[tau] + atomicAdd(&cur[tau], 1)] = t;
+  }
+}
+
+__global__ void gather_kernel(const uint4* __restrict__ X, const int* __restrict__ perm, const int* __restrict__ valid,
+                              int T, int64_t units, uint4* __restrict__ Xp) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (int64_t)T * units) return;
+  const int64_t p = e / units, u = e % units;
+  if (p >= *valid) return;
+  Xp[e] = __ldg(X + (int64_t)perm[p] * units + u);
+}
+
+}  // namespace
+
+int route_max_tiles(int64_t T, int ntask, int N) { return (int)((T + N - 1) / N) + ntask; }
+
+size_t route_workspace_bytes(int64_t T, int64_t d, int ntask, int N) {
+  const size_t words = (size_t)T + 3 * (size_t)route_max_tiles(T, ntask, N) + 1;
+  const size_t head = (words * 4 + 255) / 256 * 256;
+  return head + (size_t)T * d * 2;
+}
+
+cudaError_t launch_route(const Problem& p, const uint16_t* X, uint16_t* Y, int N, void* workspace, Routed* out,
+                         cudaStream_t s) {
+  const int max_tiles = route_max_tiles(p.T, p.ntask, N);
+  int* perm = static_cast<int*>(workspace);
+  int* tiles = perm + p.T;
+  int* valid = tiles + 3 * max_tiles;
+  const size_t words = (size_t)p.T + 3 * (size_t)max_tiles + 1;
+  uint16_t* Xp = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) + (words * 4 + 255) / 256 * 256);
+  route_kernel<<<1, kRouteThreads, 0, s>>>(p.task, (int)p.T, p.ntask, N, perm, tiles, max_tiles, valid, Y, p.n,
+                                           p.check);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t units = p.d / 8;
+  const int64_t total = p.T * units;
+  gather_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(reinterpret_cast<const uint4*>(X), perm, valid,
+                                                                (int)p.T, units, reinterpret_cast<uint4*>(Xp));
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  out->perm = perm;
+  out->tiles = tiles;
+  out->max_tiles = max_tiles;
+  out->Xp = Xp;
+  return cudaSuccess;
+}
+
+}  // namespace sk

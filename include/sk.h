@@ -122,6 +122,10 @@ sk_status sk_dequant(const void* packed, const uint16_t* lut, int bits, int gpr,
 /*
  * Workspace bytes that the call selected by `op` (SK_OP_*) needs for these
  * shapes; 0 means no workspace (a NULL workspace is then fine).
+ * SK_OP_BWD_LUT: required by the tensor-core LUT gradient (partial bins).
+ * SK_OP_FWD with ntask > 1: the task routing of the tensor-core forward
+ * (permutation, tile list and X in task order); optional -- without it a
+ * batch with several LUT sets runs on the CUDA-core kernel.
  */
 size_t sk_workspace_bytes(int op, int64_t n, int64_t d, int bits, int gpr,
                           int64_t T, int ntask);

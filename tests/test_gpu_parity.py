@@ -335,3 +335,35 @@ def test_bwd_lut_tc_workspace_required():
     st = sk.lib.sk_linear_bwd_lut(sk._ptr(packed), c.bits, c.gpr, c.n, c.d, sk._ptr(X), sk._ptr(dY), c.T, None, 1,
                                   sk._ptr(out), 0, None, 0, None)
     assert st == 1  # SK_ERR_INVALID_ARG: the tensor-core path needs its workspace
+
+
+# ---------------------------------------------------------------------------
+# several LUT sets on the tensor-core forward (task routing) and on the CUDA cores
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("path", ["auto", "gemv"])
+@pytest.mark.parametrize("T,ntask,shape", [(5, 8, (256, 1024, 4, 4)), (64, 8, (136, 512, 3, 2)),
+                                           (300, 3, (264, 1376, 2, 1)), (2048, 3, (512, 2048, 4, 4)),
+                                           (777, 8, (128, 4096, 4, 4))])
+def test_multitask_forward_each_path(monkeypatch, path, T, ntask, shape):
+    sk = _sk()
+    if path != "auto":
+        monkeypatch.setenv("SK_FWD_PATH", path)
+    n, d, bits, gpr = shape
+    c = synth.layer_case(9700 + T, n=n, d=d, bits=bits, gpr=gpr, T=T, ntask=ntask)
+    packed, lut, X, dY, task = gc.dev_case(c)
+    assert sk.workspace_bytes(sk.SK_OP_FWD, n, d, bits, gpr, T, ntask) > 0
+    gc.check_fwd(c, sk.linear_fwd(packed, lut, c.bits, X, task))
+    assert sk.device_check() == 0
+
+
+def test_multitask_forward_skewed_tasks():
+    """Most tokens on one task, a few on others, one task empty."""
+    sk = _sk()
+    c = synth.layer_case(9800, n=256, d=1024, bits=4, gpr=4, T=600, ntask=5)
+    c.task[:] = 0
+    c.task[::97] = 2
+    c.task[5] = 4
+    packed, lut, X, dY, task = gc.dev_case(c)
+    gc.check_fwd(c, sk.linear_fwd(packed, lut, c.bits, X, task))
+    assert sk.device_check() == 0
