@@ -66,11 +66,13 @@ def parse():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode7b")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--layers", default=None,
+                    help="comma-separated layer indices to run (a subset for profiling); default all")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--launch-events", choices=("auto", "on", "off"), default="auto",
-                    help="capture timing events between launches (per-kernel durations; they add "
-                         "a few microseconds per launch); auto = only when a step mixes kernels")
+    ap.add_argument("--launch-events", choices=("groups", "on", "off"), default="groups",
+                    help="timing events captured between launches: 'groups' only where the kernel "
+                         "changes (each event costs a few microseconds), 'on' between every launch")
     return ap.parse_args()
 
 
@@ -85,9 +87,15 @@ def peaks():
         return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
 
 
+_LAYER_SUBSET = None
+
+
 def layer_shapes(w):
     from compressive_fine_tuning_b200 import synth
-    return getattr(synth, w["shapes"])
+    shapes = getattr(synth, w["shapes"])
+    if _LAYER_SUBSET is not None:
+        shapes = [shapes[i] for i in _LAYER_SUBSET]
+    return shapes
 
 
 def is_hbm_bound(w):
@@ -103,6 +111,38 @@ def launch_bytes(n, d, bits, gpr, T, ntask_present=1):
 
 def launch_flops(n, d, T, op):
     return 2 * T * n * d  # each of Y, dX and the dense part of dLUT is one T x n x d contraction
+
+
+def kernel_name(op, T, w):
+    """The library kernel a launch of this kind runs (the dispatch rules of sk_api.cu)."""
+    if op == "fwd":
+        if w["ntask"] > 1:
+            return "fwd_tc_kernel (routed)"
+        return "gemv_fwd_single_kernel" if T == 1 else "fwd_tc_kernel"
+    if op == "dx":
+        return "dx_tc_kernel" if T >= 64 else "simt_bwd_input_kernel"
+    return "dlut_tc_kernel" if T >= 64 else "simt_bwd_lut_kernel"
+
+
+def traffic_per_launch(kname, workload, units_per_launch):
+    """DRAM bytes per launch from the committed ncu summary of this kernel on
+    this workload (profiles/traffic.json), scaled from the captured launch to
+    the average launch by algorithmic units; None when there is no capture or
+    any of the kernel's sources changed since the counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[f"{kname.split(' ')[0]}@{workload}"]
+        h = hashlib.sha256()
+        for name in rec["source"]:
+            with open(os.path.join(ROOT, "compressive_fine_tuning_b200", "csrc", name), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != rec["source_sha256"]:
+            return None
+        return rec["dram_bytes"] * units_per_launch / rec["algorithmic_units"]
+    except Exception:
+        return None
 
 
 # ---------------------------------------------------------------------------
@@ -280,8 +320,6 @@ def run_ours(args, w, rank, world, device):
 
     stream = torch.cuda.Stream(device)
     K, W = args.steps, args.warmup
-    if args.launch_events == "auto":
-        args.launch_events = "off" if len(w["ops"]) == 1 else "on"
 
     # warm-up (eager), also the first-call setup of every kernel
     with torch.cuda.stream(stream):
@@ -290,17 +328,27 @@ def run_ours(args, w, rank, world, device):
                 launch(li, T, op, s)
     torch.cuda.synchronize(device)
 
-    # capture one graph per timed step, with external timing events between launches
+    # event boundaries: before the first launch, then wherever the kernel type
+    # (op, token count) changes, and after the last launch
+    kinds = [(op, T) for (li, T, op, u) in plan]
+    if args.launch_events == "on":
+        bounds = list(range(len(plan) + 1))
+    elif args.launch_events == "groups":
+        bounds = [0] + [j for j in range(1, len(plan)) if kinds[j] != kinds[j - 1]] + [len(plan)]
+    else:
+        bounds = []
+
+    # capture one graph per timed step, with external timing events at the boundaries
     graphs, ev = [], []
     for s in range(K):
         g = torch.cuda.CUDAGraph()
-        evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(plan) + 1)]
+        evs = {b: torch.cuda.Event(enable_timing=True, external=True) for b in bounds}
         with torch.cuda.graph(g, stream=stream):
-            if args.launch_events == "on":
+            if 0 in evs:
                 evs[0].record()
             for j, (li, T, op, u) in enumerate(plan):
                 launch(li, T, op, W + s)
-                if args.launch_events == "on":
+                if j + 1 in evs:
                     evs[j + 1].record()
         graphs.append(g)
         ev.append(evs)
@@ -332,18 +380,18 @@ def run_ours(args, w, rank, world, device):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
 
-    # per-launch durations from the captured events (without them: the step
-    # time spread over the launches in proportion to their units)
-    if args.launch_events == "on":
-        per_launch = np.array([[ev[s][j].elapsed_time(ev[s][j + 1]) for j in range(len(plan))] for s in range(K)])
-        launches_ms = per_launch.sum(axis=0) / K  # mean per launch position
+    # time per kernel type: groups of launches between boundary events; without
+    # events the step time is spread over the launches in proportion to units
+    groups = []   # (kind, units, ms per step)
+    if bounds:
+        for a0, a1 in zip(bounds[:-1], bounds[1:]):
+            t = sum(ev[s][a0].elapsed_time(ev[s][a1]) for s in range(K)) / K
+            groups.append((kinds[a0], sum(p[3] for p in plan[a0:a1]), t, a1 - a0))
     else:
-        u = np.array([p[3] for p in plan], dtype=np.float64)
-        launches_ms = (ms / K) * u / u.sum()
-
+        groups.append((kinds[0], step_units, ms / K, len(plan)))
     total_units = step_units * K * world
     value = total_units / (ms / 1e3)
-    res = dict(ms=ms, value=value, plan=plan, per_launch_ms=launches_ms, step_units=step_units,
+    res = dict(ms=ms, value=value, plan=plan, groups=groups, step_units=step_units,
                hbm_bound=hbm_bound, clocks=clocks, copies=copies, weight_bytes=weight_bytes)
 
     # end-to-end through the public API with host buffers (one rank's view)
@@ -404,8 +452,11 @@ def fmt_units(w):
 
 
 def main():
+    global _LAYER_SUBSET
     args = parse()
     w = WORKLOADS[args.workload]
+    if args.layers:
+        _LAYER_SUBSET = [int(x) for x in args.layers.split(",")]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -414,7 +465,8 @@ def main():
     config = {"workload": args.workload, "desc": w["desc"], "bits": w["bits"], "gpr": w["gpr"],
               "tokens": list(w["batches"]), "ntask": w["ntask"], "layers": [list(s) for s in layer_shapes(w)],
               "parallelism": f"replicas{args.gpus}" if args.gpus > 1 else "single",
-              "l2": "weights rotate over copies totalling > 3x L2"}
+              "l2": "weights rotate over copies totalling > 3x L2",
+              "layer_subset": _LAYER_SUBSET}
 
     if args.impl == "reference":
         if rank != 0:
@@ -450,33 +502,36 @@ def main():
     if rank != 0:
         return 0
 
-    plan = res["plan"]
-    per = res["per_launch_ms"]
+    # the dominant kernel: the kernel type (op, tokens) with the largest share of
+    # the step; its achieved rate = its algorithmic units / its measured time
+    by_kind = {}
+    for kind, units, t, nl in res["groups"]:
+        a = by_kind.setdefault(kind, [0.0, 0.0, 0])
+        a[0] += units; a[1] += t; a[2] += nl
+    dom = max(by_kind, key=lambda k: by_kind[k][1])
+    units, t_ms, nl = by_kind[dom]
+    step_ms = res["ms"] / args.steps
+    op, T = dom
+    kname = kernel_name(op, T, w)
     if res["hbm_bound"]:
-        dom_units = sum(p[3] for p in plan)
-        dom_ms = float(per.sum())
-        achieved = dom_units / (dom_ms / 1e3) / 1e9
+        achieved = units / (t_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
-                "frac": achieved / pk["hbm"], "traffic": None, "kernel": "sk_linear_fwd (LUT-GEMV)",
-                "peak_source": pk["source"] + " hbm_gbs (copy)",
-                "per_launch_us": [round(x * 1e3, 2) for x in per]}
+                "frac": achieved / pk["hbm"], "traffic": traffic_per_launch(kname, args.workload, units / max(nl, 1)),
+                "kernel": kname, "launches_per_step": nl, "share": t_ms / step_ms,
+                "peak_source": pk["source"] + " hbm_gbs (copy)"}
     else:
-        # the dominant kernel: the op with the largest total time
-        by_op = {}
-        for (li, T, op, u), t in zip(plan, per):
-            a = by_op.setdefault(op, [0.0, 0.0])
-            a[0] += u; a[1] += t
-        op = max(by_op, key=lambda o: by_op[o][1])
-        achieved = by_op[op][0] / (by_op[op][1] / 1e3) / 1e12
+        achieved = units / (t_ms / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_sus"], "unit": "TFLOP/s",
-                "frac": achieved / pk["bf16_sus"], "traffic": None, "kernel": op,
-                "peak_source": pk["source"] + " bf16_tflops_sustained",
-                "by_op_tflops": {o: v[0] / (v[1] / 1e3) / 1e12 for o, v in by_op.items()}}
+                "frac": achieved / pk["bf16_sus"], "traffic": traffic_per_launch(kname, args.workload, units / max(nl, 1)),
+                "kernel": kname, "launches_per_step": nl, "share": t_ms / step_ms,
+                "peak_source": pk["source"] + " bf16_tflops_sustained (a kernel timed inside a long step)"}
+    roof["by_kernel"] = {f"{kernel_name(k[0], k[1], w)} T={k[1]}": {
+        "rate": v[0] / (v[1] / 1e3) / scale, "unit": unit, "share": v[1] / step_ms} for k, v in by_kind.items()}
 
     line = {"metric": METRIC, "value": res["value"] / scale, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": res["ms"] / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config,
-            "roofline": roof, "gpu_launches": len(plan) * args.steps,
+            "roofline": roof, "gpu_launches": len(res["plan"]) * args.steps,
             "clocks": res["clocks"]}
     if "e2e" in res:
         e = res["e2e"]
