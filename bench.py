@@ -12,6 +12,11 @@ Other workloads (--workload) time the training products (forward, input
 gradient and LUT gradient per layer) in TFLOP/s and the 70B multi-task
 serving shapes; they print the same JSON contract.
 
+Multi-GPU (torchrun, one process per GPU): decode and serving run as
+independent replicas; the training workloads run data-parallel, each rank on
+its own token batch, with one NCCL all-reduce of the fp32 LUT gradient per
+layer on a side stream.  Both scale weakly.
+
 Timing: W warm-up steps, then K steps captured as CUDA graphs and replayed back
 to back, bracketed by a barrier and a device synchronisation on each side,
 timed with CUDA events on the launching stream; multi-GPU runs take the max
@@ -122,6 +127,17 @@ def kernel_name(op, T, w):
     if op == "dx":
         return "dx_tc_kernel" if T >= 64 else "simt_bwd_input_kernel"
     return "dlut_tc_kernel" if T >= 64 else "simt_bwd_lut_kernel"
+
+
+def kernels_per_launch(op, T, w):
+    """Library kernels one API call of this kind launches: the routed forward
+    adds the routing and gather kernels, the tensor-core LUT gradient adds its
+    reduction of partial bins."""
+    if op == "fwd" and w["ntask"] > 1:
+        return 3
+    if op == "dlut" and T >= 64:
+        return 2
+    return 1
 
 
 def traffic_per_launch(kname, workload, units_per_launch):
@@ -318,14 +334,35 @@ def run_ours(args, w, rank, world, device):
         else:
             sk.linear_bwd_lut(packed, bits, gpr, a["X"], a["dY"], a["task"], ntask, out=a["dl"])
 
+    # data-parallel fine-tuning: every rank runs its own T tokens (weak
+    # scaling) and the LUT gradients are summed over ranks, one all-reduce per
+    # layer on a side stream, joined at the end of the step
+    reducer = None
+    if world > 1 and "dlut" in w["ops"]:
+        from compressive_fine_tuning_b200 import dp
+        reducer = dp.LutGradReducer()
+
+    def after(op, li, T):
+        if reducer is not None and op == "dlut":
+            reducer.submit(acts[(li, T)]["dl"])
+
+    def end_step():
+        if reducer is not None:
+            reducer.wait()
+
     stream = torch.cuda.Stream(device)
     K, W = args.steps, args.warmup
+    # NCCL calls are issued eagerly (no graph capture) so that every rank's
+    # collectives stay in plain stream order
+    use_graphs = reducer is None
 
     # warm-up (eager), also the first-call setup of every kernel
     with torch.cuda.stream(stream):
         for s in range(W):
             for (li, T, op, u) in plan:
                 launch(li, T, op, s)
+                after(op, li, T)
+            end_step()
     torch.cuda.synchronize(device)
 
     # event boundaries: before the first launch, then wherever the kernel type
@@ -338,19 +375,25 @@ def run_ours(args, w, rank, world, device):
     else:
         bounds = []
 
+    def record_step(s, evs):
+        if 0 in evs:
+            evs[0].record()
+        for j, (li, T, op, u) in enumerate(plan):
+            launch(li, T, op, W + s)
+            after(op, li, T)
+            if j + 1 in evs:
+                evs[j + 1].record()
+        end_step()
+
     # capture one graph per timed step, with external timing events at the boundaries
     graphs, ev = [], []
     for s in range(K):
-        g = torch.cuda.CUDAGraph()
-        evs = {b: torch.cuda.Event(enable_timing=True, external=True) for b in bounds}
-        with torch.cuda.graph(g, stream=stream):
-            if 0 in evs:
-                evs[0].record()
-            for j, (li, T, op, u) in enumerate(plan):
-                launch(li, T, op, W + s)
-                if j + 1 in evs:
-                    evs[j + 1].record()
-        graphs.append(g)
+        evs = {b: torch.cuda.Event(enable_timing=True, external=use_graphs) for b in bounds}
+        if use_graphs:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                record_step(s, evs)
+            graphs.append(g)
         ev.append(evs)
     torch.cuda.synchronize(device)
     for g in graphs[:2]:  # replay warm-up
@@ -367,8 +410,12 @@ def run_ours(args, w, rank, world, device):
     torch.cuda.synchronize(device)
     with torch.cuda.stream(stream):
         start.record(stream)
-        for g in graphs:
-            g.replay()
+        if use_graphs:
+            for g in graphs:
+                g.replay()
+        else:
+            for s in range(K):
+                record_step(s, ev[s])
         stop.record(stream)
     torch.cuda.synchronize(device)
     if world > 1:
@@ -434,6 +481,9 @@ def run_ours(args, w, rank, world, device):
                         out = sk.linear_bwd_input(packed, lut, bits, L["d"], dY, tk)
                     else:
                         out = sk.linear_bwd_lut(packed, bits, gpr, X, dY, tk, ntask)
+                    if reducer is not None and op == "dlut":
+                        reducer.submit(out)
+                        reducer.wait()
                     hb["out"][{"fwd": "Y", "dx": "dX", "dlut": "dl"}[op]].copy_(out, non_blocking=True)
             e1.record(stream)
         torch.cuda.synchronize(device)
@@ -464,7 +514,9 @@ def main():
     pk = peaks()
     config = {"workload": args.workload, "desc": w["desc"], "bits": w["bits"], "gpr": w["gpr"],
               "tokens": list(w["batches"]), "ntask": w["ntask"], "layers": [list(s) for s in layer_shapes(w)],
-              "parallelism": f"replicas{args.gpus}" if args.gpus > 1 else "single",
+              "parallelism": ("single" if world == 1 else
+                              f"dp{world} (tokens per rank; LUT-gradient all-reduce)" if "dlut" in w["ops"]
+                              else f"replicas{world}"),
               "l2": "weights rotate over copies totalling > 3x L2",
               "layer_subset": _LAYER_SUBSET}
 
@@ -531,7 +583,7 @@ def main():
     line = {"metric": METRIC, "value": res["value"] / scale, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": res["ms"] / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config,
-            "roofline": roof, "gpu_launches": len(res["plan"]) * args.steps,
+            "roofline": roof, "gpu_launches": sum(kernels_per_launch(op, T, w) for (_, T, op, _) in res["plan"]) * args.steps,
             "clocks": res["clocks"]}
     if "e2e" in res:
         e = res["e2e"]
