@@ -123,7 +123,12 @@ def kernel_name(op, T, w):
     if op == "fwd":
         if w["ntask"] > 1:
             return "fwd_tc_kernel (routed)"
-        return "gemv_fwd_single_kernel" if T == 1 else "fwd_tc_kernel"
+        path = os.environ.get("SK_FWD_PATH", "")
+        if w["bits"] == 4 and T <= 16 and path not in ("gemv", "tc"):
+            return "decode_kernel"
+        if path == "gemv" or (T == 1 and path != "tc"):
+            return "gemv_fwd_single_kernel"
+        return "fwd_tc_kernel"
     if op == "dx":
         return "dx_tc_kernel" if T >= 64 else "simt_bwd_input_kernel"
     return "dlut_tc_kernel" if T >= 64 else "simt_bwd_lut_kernel"

@@ -82,10 +82,11 @@ size_t row_bytes(int64_t d, int bits) {
 
 constexpr int64_t kMaxDim = int64_t(1) << 31;
 
-// Kernel choice for the forward.  SK_FWD_PATH=gemv|tc forces one path (for
-// measurements and tests); by default the tensor-core kernel takes every
-// single-LUT-set batch of at least kFwdTcMinT tokens on layers at least 128
-// columns wide.
+// Kernel choice for the forward.  SK_FWD_PATH=gemv|tc|dq forces one path (for
+// measurements and tests).  By default a single-LUT-set batch runs on the
+// decode kernel when it applies (4-bit, T <= 16), else on the tensor-core
+// kernel from kFwdTcMinT tokens on layers at least 128 columns wide, else on
+// the CUDA-core kernel.
 constexpr int64_t kFwdTcMinT = 2;
 
 int env_path(const char* name) {
@@ -93,6 +94,7 @@ int env_path(const char* name) {
   if (v == nullptr) return 0;
   if (strcmp(v, "gemv") == 0 || strcmp(v, "simt") == 0) return 1;
   if (strcmp(v, "tc") == 0) return 2;
+  if (strcmp(v, "dq") == 0) return 3;
   return 0;
 }
 
@@ -115,6 +117,12 @@ bool use_tensor_cores_fwd(const sk::Problem& p) {
   if (forced == 1) return false;
   if (forced == 2) return tc_ok;
   return tc_ok && p.T >= kFwdTcMinT;
+}
+
+bool use_decode_fwd(const sk::Problem& p) {
+  const int forced = env_path("SK_FWD_PATH");
+  if (forced == 1 || forced == 2) return false;
+  return sk::decode_fwd_supported(p);
 }
 
 // Several LUT sets: the tensor-core forward needs the routing workspace.
@@ -291,7 +299,9 @@ sk_status sk_linear_fwd(const void* packed, const uint16_t* lut, int bits, int g
       e = sk::launch_gemv_fwd(p, X, Y, s);
     }
   } else {
-    e = use_tensor_cores_fwd(p) ? sk::launch_fwd_tc(p, X, Y, s) : sk::launch_gemv_fwd(p, X, Y, s);
+    e = use_decode_fwd(p)         ? sk::launch_decode_fwd(p, X, Y, s)
+        : use_tensor_cores_fwd(p) ? sk::launch_fwd_tc(p, X, Y, s)
+                                  : sk::launch_gemv_fwd(p, X, Y, s);
   }
   return e == cudaSuccess ? ok() : cuda_fail(e, "forward kernel launch");
 }

@@ -337,6 +337,9 @@ cudaError_t launch_unpack(const uint8_t* packed, int64_t n, int64_t d, int bits,
                           uint8_t* idx, cudaStream_t s);
 cudaError_t launch_dequant(const Problem& p, int task, uint16_t* theta, cudaStream_t s);
 cudaError_t launch_gemv_fwd(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStream_t s);
+// Decode forward (4-bit, single LUT set, 1 <= T <= 16, d >= 256) on mma.sync.
+bool decode_fwd_supported(const Problem& p);
+cudaError_t launch_decode_fwd(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStream_t s);
 cudaError_t launch_fwd_tc(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStream_t s);
 cudaError_t launch_dx_tc(const Problem& p, const uint16_t* dY, uint16_t* dX, cudaStream_t s);
 cudaError_t launch_dlut_tc(const Problem& p, const uint16_t* X, const uint16_t* dY, float* dlut, int accumulate,

@@ -105,6 +105,14 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// 3-D tile load: coordinates (x innermost, y, z); x * elemsize % 16 == 0.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
 // ----------------------------------------------------------------------------
 // tensor memory
 // ----------------------------------------------------------------------------
@@ -243,6 +251,13 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 cudaError_t make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem_bytes,
                          uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
                          uint32_t box_outer, CUtensorMapSwizzle swizzle);
+
+// 3-D tensor map: dims[0] contiguous elements, dims[1] and dims[2] at byte
+// strides stride1 and stride2 (multiples of 16, in any order); box of
+// box0 x box1 x box2 elements.
+cudaError_t make_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, uint64_t dim0,
+                         uint64_t dim1, uint64_t dim2, uint64_t stride1, uint64_t stride2, uint32_t box0,
+                         uint32_t box1, uint32_t box2, CUtensorMapSwizzle swizzle);
 
 // Launch attributes shared by the tensor-core kernels.
 int num_sms();

@@ -1,0 +1,99 @@
+"""Parity of the decode forward kernel (4-bit, one LUT set, 1 <= T <= 16) with the oracle.
+
+The decode kernel splits the rows over the CTAs (several 16-row tiles per CTA
+once the layer has more tiles than the GPU has SMs), streams the columns in
+stages of 512 to 2048 columns, and permutes the K order inside every MMA
+step.  The shapes
+below make each of those visible: ragged last row tiles, a partial last stage,
+groups that straddle stages, 32-column groups, CTAs whose warps span two row
+tiles, and token counts on both sides of the 8-token MMA tile.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+from compressive_fine_tuning_b200 import synth  # noqa: E402
+from tests import gpu_cases as gc  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from compressive_fine_tuning_b200 import sk  # noqa: F401
+    yield
+    torch.cuda.synchronize()
+
+
+DECODE_SHAPES = [
+    (256, 512, 1),      # the tiny configuration, one stage
+    (4104, 4096, 8),    # 257 row tiles: two per CTA, ragged last tile
+    (2376, 2816, 2),    # 1408-column groups straddling stages, partial last stage
+    (96, 512, 16),      # 32-column groups, many per stage
+    (264, 256, 1),      # narrowest width the kernel takes, one 256-column block
+]
+
+
+@pytest.mark.parametrize("shape", DECODE_SHAPES)
+@pytest.mark.parametrize("T", [1, 2, 5, 8, 9, 16])
+def test_decode_forward(monkeypatch, shape, T):
+    from compressive_fine_tuning_b200 import sk
+    monkeypatch.setenv("SK_FWD_PATH", "dq")
+    n, d, gpr = shape
+    c = synth.layer_case(31000 + n + T, n=n, d=d, bits=4, gpr=gpr, T=T)
+    packed, lut, X, dY, task = gc.dev_case(c)
+    Y = sk.linear_fwd(packed, lut, 4, X, task)
+    gc.check_fwd(c, Y)
+    assert sk.device_check() == 0
+
+
+@pytest.mark.parametrize("n,d", [(11008, 4096), (4096, 11008)])
+@pytest.mark.parametrize("T", [1, 16])
+def test_decode_forward_7b_shapes(monkeypatch, n, d, T):
+    """The gate/up shape puts four or five row tiles in every CTA, so a warp's
+    items span two row tiles; the down shape ends on a 256-column stage."""
+    from compressive_fine_tuning_b200 import sk
+    monkeypatch.setenv("SK_FWD_PATH", "dq")
+    c = synth.layer_case(32000 + n + T, n=n, d=d, bits=4, gpr=8, T=T)
+    packed, lut, X, dY, task = gc.dev_case(c)
+    Y = sk.linear_fwd(packed, lut, 4, X, task)
+    gc.check_fwd(c, Y)
+    assert sk.device_check() == 0
+
+
+@pytest.mark.parametrize("T", [1, 16])
+def test_decode_matches_tensor_core_path_and_is_deterministic(monkeypatch, T):
+    """Both kernels round the same bf16 weights; fp32 sums in different orders
+    agree to a few bf16 ulps, and the decode kernel repeats itself bit for bit."""
+    from compressive_fine_tuning_b200 import sk
+    c = synth.layer_case(33000 + T, n=4096, d=4096, bits=4, gpr=8, T=T)
+    packed, lut, X, dY, task = gc.dev_case(c)
+    monkeypatch.setenv("SK_FWD_PATH", "dq")
+    y1 = sk.linear_fwd(packed, lut, 4, X, task)
+    y2 = sk.linear_fwd(packed, lut, 4, X, task)
+    assert torch.equal(y1, y2)
+    monkeypatch.setenv("SK_FWD_PATH", "tc")
+    y3 = sk.linear_fwd(packed, lut, 4, X, task)
+    a, b = y1.float(), y3.float()
+    assert torch.allclose(a, b, rtol=2 ** -6, atol=1e-3 * b.abs().max().item())
+
+
+def test_decode_identity_is_exact(monkeypatch):
+    """idx = I with the {0, 1} LUT (SpaLLM section 2.4): Y == X bit for bit."""
+    from compressive_fine_tuning_b200 import sk
+    monkeypatch.setenv("SK_FWD_PATH", "dq")
+    n = d = 512
+    idx = np.zeros((n, d), dtype=np.uint8)
+    idx[np.arange(n), np.arange(n)] = 1
+    lut = np.zeros((1, n, 1, 16), dtype=np.float16)
+    lut[..., 1] = 1.0
+    lut[..., 2:] = np.float16(np.nan)   # never read
+    rng = synth.rng_for(34000)
+    x = synth.make_bf16(rng, (7, d), 1.0)
+    packed = sk.pack(torch.from_numpy(idx).cuda(), 4)
+    X = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+    Y = sk.linear_fwd(packed, torch.from_numpy(lut).cuda(), 4, X, None)
+    np.testing.assert_array_equal(Y.view(torch.int16).cpu().numpy().view(np.uint16), x)

@@ -274,7 +274,7 @@ def fwd_path(monkeypatch):
     yield set_path
 
 
-@pytest.mark.parametrize("path", ["tc", "gemv"])
+@pytest.mark.parametrize("path", ["tc", "gemv", "dq"])
 @pytest.mark.parametrize("shape", [(256, 512, 4, 1), (136, 320, 2, 5), (264, 1376, 3, 1), (1024, 4096, 4, 8)])
 @pytest.mark.parametrize("T", [1, 2, 17, 64, 129])
 def test_forward_each_path(fwd_path, path, shape, T):
