@@ -61,6 +61,10 @@ WORKLOADS = {
 }
 
 L2_BYTES = 126 * 1024 * 1024
+# Integer-ALU cost of one 4-bit lookup (byte-permute network) and the integer
+# pipe's issue rate per SM on B200, measured with a throughput probe.
+ALU_OPS_PER_4BIT_WEIGHT = 2.25
+INT_LANES_PER_SM = 64
 
 
 def parse():
@@ -582,6 +586,19 @@ def main():
                 "frac": achieved / pk["bf16_sus"], "traffic": traffic_per_launch(kname, args.workload, units / max(nl, 1)),
                 "kernel": kname, "launches_per_step": nl, "share": t_ms / step_ms,
                 "peak_source": pk["source"] + " bf16_tflops_sustained (a kernel timed inside a long step)"}
+    if res["hbm_bound"] and kname == "decode_kernel" and w["bits"] == 4:
+        # The decode kernel is bound by the integer pipe, not by HBM: every 4-bit
+        # weight costs 2.25 integer-ALU lane operations at least (16 byte permutes
+        # and 2 masks per eight weights), and the integer pipe issues 64 lanes per
+        # cycle per SM on this GPU (measured).  Reported beside the HBM roofline.
+        shapes = layer_shapes(w)
+        lookups = sum(shapes[li][0] * shapes[li][1] for (li, T_, op_, u_) in res["plan"] if (op_, T_) == dom)
+        mhz = (res["clocks"] or {}).get("sm_mhz") or 1965.0
+        ops = lookups * ALU_OPS_PER_4BIT_WEIGHT / (t_ms / 1e3)
+        alu_peak = torch.cuda.get_device_properties(device).multi_processor_count * INT_LANES_PER_SM * mhz * 1e6
+        roof["alu"] = {"achieved": ops / 1e12, "peak": alu_peak / 1e12, "unit": "T int-lane-ops/s",
+                       "frac": ops / alu_peak, "ops_per_weight": ALU_OPS_PER_4BIT_WEIGHT,
+                       "peak_source": f"{INT_LANES_PER_SM} integer lanes/cycle/SM (measured) x SMs x median SM clock"}
     roof["by_kernel"] = {f"{kernel_name(k[0], k[1], w)} T={k[1]}": {
         "rate": v[0] / (v[1] / 1e3) / scale, "unit": unit, "share": v[1] / step_ms} for k, v in by_kind.items()}
 
