@@ -295,43 +295,99 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constant__
               x1[nt] = lds128(xc + x_lane[nt] + 64);
             }
           };
-          // with 8 consumer warps the next pair's operands are loaded before this
-          // pair's lookups, so their shared-memory latency hides behind the
-          // permutes; 16 warps hide it by switching warps and keep the registers
-          uint32_t wc[4];
-          uint4 xc0[NT], xc1[NT];
-          fetch(cb, wc, xc0, xc1);
-#pragma unroll 2
-          for (int c = cb; c < ce; c += 2) {
-            uint32_t wn[4];
-            uint4 xn0[NT], xn1[NT];
-            if constexpr (PIPE) fetch(c + 2 < ce ? c + 2 : c, wn, xn0, xn1);
-            const int col = k0 + 32 * c;
-            if (!one_group && col >= gend) { do { ++g; gend += gs32; } while (col >= gend); planes_for(g); }
+          // lookups and MMAs of one chunk pair from its fetched operands
+          auto pair_body = [&](const uint32_t (&w)[4], const uint4 (&x0)[NT], const uint4 (&x1)[NT], bool planes_change,
+                               int col) {
             uint32_t af0[2][4];
-            dequant_frags(wc[0], wc[1], lo0, hi0, lo1, hi1, af0);
+            dequant_frags(w[0], w[1], lo0, hi0, lo1, hi1, af0);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-              mma_bf16_16816(acc[0][0][nt], af0[0], xc0[nt].x, xc0[nt].y);
-              mma_bf16_16816(acc[0][CH - 1][nt], af0[1], xc0[nt].z, xc0[nt].w);
+              mma_bf16_16816(acc[0][0][nt], af0[0], x0[nt].x, x0[nt].y);
+              mma_bf16_16816(acc[0][CH - 1][nt], af0[1], x0[nt].z, x0[nt].w);
             }
-            if (c + 1 < ce) {
-              if (!one_group && col + 32 >= gend) { ++g; gend += gs32; planes_for(g); }
-              uint32_t af1[2][4];
-              dequant_frags(wc[2], wc[3], lo0, hi0, lo1, hi1, af1);
+            if (planes_change && col + 32 >= gend) { ++g; gend += gs32; planes_for(g); }  // boundary inside the pair
+            uint32_t af1[2][4];
+            dequant_frags(w[2], w[3], lo0, hi0, lo1, hi1, af1);
 #pragma unroll
-              for (int nt = 0; nt < NT; ++nt) {
-                mma_bf16_16816(acc[1][0][nt], af1[0], xc1[nt].x, xc1[nt].y);
-                mma_bf16_16816(acc[1][CH - 1][nt], af1[1], xc1[nt].z, xc1[nt].w);
+            for (int nt = 0; nt < NT; ++nt) {
+              mma_bf16_16816(acc[1][0][nt], af1[0], x1[nt].x, x1[nt].y);
+              mma_bf16_16816(acc[1][CH - 1][nt], af1[1], x1[nt].z, x1[nt].w);
+            }
+          };
+          // without the software pipeline: the X fragments of the pair's second
+          // chunk are loaded after the first chunk's MMAs (fewer live registers)
+          auto x_addr = [&](int c) { return xs + (uint32_t)(c >> 3) * x_box + ((uint32_t)(c & 7) << 6); };
+          auto fetch_lazy = [&](int c, uint32_t (&w)[4], uint4 (&x0)[NT]) {
+            const uint32_t addr = idx_row + (uint32_t)(c >> 3) * box_stride +
+                                  ((((uint32_t)(c & 7) + (uint32_t)lm_chunk) ^ lm_x) << 4);
+            asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(addr));
+            const uint32_t xc = x_addr(c);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) x0[nt] = lds128(xc + x_lane[nt]);
+          };
+          auto pair_body_lazy = [&](int c, const uint32_t (&w)[4], const uint4 (&x0)[NT], bool planes_change = false,
+                                    int col = 0) {
+            uint32_t af0[2][4];
+            dequant_frags(w[0], w[1], lo0, hi0, lo1, hi1, af0);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              mma_bf16_16816(acc[0][0][nt], af0[0], x0[nt].x, x0[nt].y);
+              mma_bf16_16816(acc[0][CH - 1][nt], af0[1], x0[nt].z, x0[nt].w);
+            }
+            if (planes_change && col + 32 >= gend) { ++g; gend += gs32; planes_for(g); }
+            uint4 x1[NT];
+            const uint32_t xc = x_addr(c) + 64;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) x1[nt] = lds128(xc + x_lane[nt]);
+            uint32_t af1[2][4];
+            dequant_frags(w[2], w[3], lo0, hi0, lo1, hi1, af1);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              mma_bf16_16816(acc[1][0][nt], af1[0], x1[nt].x, x1[nt].y);
+              mma_bf16_16816(acc[1][CH - 1][nt], af1[1], x1[nt].z, x1[nt].w);
+            }
+          };
+          // d % 256 == 0, so every run is whole chunk pairs.  A run inside one
+          // group (the usual case) has no checks in its loop.  With 8 consumer
+          // warps the next pair's operands are loaded before this pair's
+          // lookups, so their shared-memory latency hides behind the permutes;
+          // 16 warps hide it by switching warps and keep the registers.
+          uint32_t wc[4];
+          uint4 xc0[NT], xc1[NT];
+          if (one_group) {
+            if constexpr (PIPE) {
+              fetch(cb, wc, xc0, xc1);
+#pragma unroll 2
+              for (int c = cb; c < ce; c += 2) {
+                uint32_t wn[4];
+                uint4 xn0[NT], xn1[NT];
+                fetch(c + 2 < ce ? c + 2 : c, wn, xn0, xn1);
+                pair_body(wc, xc0, xc1, false, 0);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) wc[k] = wn[k];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) { xc0[nt] = xn0[nt]; xc1[nt] = xn1[nt]; }
+              }
+            } else {
+#pragma unroll 2
+              for (int c = cb; c < ce; c += 2) {
+                fetch_lazy(c, wc, xc0);
+                pair_body_lazy(c, wc, xc0);
               }
             }
-            if constexpr (PIPE) {
-#pragma unroll
-              for (int k = 0; k < 4; ++k) wc[k] = wn[k];
-#pragma unroll
-              for (int nt = 0; nt < NT; ++nt) { xc0[nt] = xn0[nt]; xc1[nt] = xn1[nt]; }
-            } else if (c + 2 < ce) {
-              fetch(c + 2, wc, xc0, xc1);
+          } else {
+#pragma unroll 1
+            for (int c = cb; c < ce; c += 2) {
+              const int col = k0 + 32 * c;
+              if (col >= gend) { do { ++g; gend += gs32; } while (col >= gend); planes_for(g); }
+              if constexpr (PIPE) {
+                fetch(c, wc, xc0, xc1);
+                pair_body(wc, xc0, xc1, true, col);
+              } else {
+                fetch_lazy(c, wc, xc0);
+                pair_body_lazy(c, wc, xc0, true, col);
+              }
             }
           }
           if (r) { grB = g; grB_end = gend; } else { grA = g; grA_end = gend; }
