@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
+#include <cmath>
 #include <cstring>
 #include <string>
 
@@ -408,6 +409,83 @@ sk_status sk_linear_bwd_lut_noalloc(const void* packed, int bits, int gpr, int64
     e = sk::launch_simt_bwd_lut(p, X, dY, dlut, accumulate, s);
   }
   return e == cudaSuccess ? ok() : cuda_fail(e, "LUT-gradient kernel launch");
+}
+
+sk_status sk_bin_counts(const void* packed, int bits, int gpr, int64_t n, int64_t d, int32_t* counts,
+                        sk_stream_t stream) {
+  g_last_error.clear();
+  sk_status st = check_shape(bits, gpr, n, d, 0, 1);
+  if (st != SK_OK) return st;
+  if (!packed || !counts) return fail(SK_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(packed) || !aligned16(counts)) return fail(SK_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  const size_t cb = (size_t)n * gpr * (1u << bits) * 4;
+  if (overlaps(counts, cb, packed, sk_packed_bytes(n, d, bits))) return fail(SK_ERR_INVALID_ARG, "output overlaps an input");
+  unsigned int* check = nullptr;
+  st = device_state(&check);
+  if (st != SK_OK) return st;
+  cudaError_t e = sk::launch_bin_counts(static_cast<const uint8_t*>(packed), (int64_t)sk_packed_row_bytes(d, bits), bits,
+                                        n, gpr, d / gpr, counts, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ok() : cuda_fail(e, "bin-count kernel launch");
+}
+
+// Checks shared by the LUT updates: sizes, pointers, and that no output
+// overlaps another buffer.
+static sk_status check_update(const void* const* outs, int nout, const float* grad, const int32_t* counts, int ntask,
+                              int64_t n, int gpr, int bits, int64_t* total, int64_t* per_set) {
+  if (bits < 2 || bits > 4) return fail(SK_ERR_INVALID_ARG, "bits must be 2, 3 or 4 (got %d)", bits);
+  if (ntask < 1 || n < 1 || gpr < 1 || n >= kMaxDim || gpr >= (1 << 24))
+    return fail(SK_ERR_INVALID_ARG, "ntask, n and gpr must be positive");
+  *per_set = n * gpr * (1 << bits);
+  *total = *per_set * ntask;
+  const size_t fb = (size_t)*total * 4, hb = (size_t)*total * 2, cb = (size_t)*per_set * 4;
+  if (!grad) return fail(SK_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(grad) || (counts && !aligned16(counts))) return fail(SK_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  for (int a = 0; a < nout; ++a) {
+    const bool half = a == nout - 1;            // the last output is the fp16 LUT (may be NULL)
+    if (!outs[a] && !half) return fail(SK_ERR_INVALID_ARG, "null pointer");
+    if (!outs[a]) continue;
+    if (!aligned16(outs[a])) return fail(SK_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+    const size_t ab = half ? hb : fb;
+    if (overlaps(outs[a], ab, grad, fb) || (counts && overlaps(outs[a], ab, counts, cb)))
+      return fail(SK_ERR_INVALID_ARG, "output overlaps an input");
+    for (int b = 0; b < a; ++b)
+      if (outs[b] && overlaps(outs[a], ab, outs[b], fb)) return fail(SK_ERR_INVALID_ARG, "outputs overlap");
+  }
+  return SK_OK;
+}
+
+sk_status sk_lut_adamw(float* master, float* m, float* v, const float* grad, const int32_t* counts, int ntask,
+                       int64_t n, int gpr, int bits, float lr, float beta1, float beta2, float eps,
+                       float weight_decay, int step, uint16_t* lut, sk_stream_t stream) {
+  g_last_error.clear();
+  const void* outs[4] = {master, m, v, lut};
+  int64_t total = 0, per_set = 0;
+  sk_status st = check_update(outs, 4, grad, counts, ntask, n, gpr, bits, &total, &per_set);
+  if (st != SK_OK) return st;
+  if (!(std::isfinite(lr) && beta1 >= 0.f && beta1 < 1.f && beta2 >= 0.f && beta2 < 1.f && eps > 0.f &&
+        std::isfinite(eps) && std::isfinite(weight_decay) && step >= 1))
+    return fail(SK_ERR_INVALID_ARG, "AdamW needs finite lr and weight_decay, 0 <= beta < 1, eps > 0, step >= 1");
+  unsigned int* check = nullptr;
+  st = device_state(&check);
+  if (st != SK_OK) return st;
+  cudaError_t e = sk::launch_adamw(master, m, v, grad, counts, total, per_set, lr, beta1, beta2, eps, weight_decay,
+                                   step, lut, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ok() : cuda_fail(e, "AdamW kernel launch");
+}
+
+sk_status sk_lut_sgd(float* master, const float* grad, const int32_t* counts, int ntask, int64_t n, int gpr,
+                     int bits, float lr, uint16_t* lut, sk_stream_t stream) {
+  g_last_error.clear();
+  const void* outs[2] = {master, lut};
+  int64_t total = 0, per_set = 0;
+  sk_status st = check_update(outs, 2, grad, counts, ntask, n, gpr, bits, &total, &per_set);
+  if (st != SK_OK) return st;
+  if (!std::isfinite(lr)) return fail(SK_ERR_INVALID_ARG, "lr must be finite");
+  unsigned int* check = nullptr;
+  st = device_state(&check);
+  if (st != SK_OK) return st;
+  cudaError_t e = sk::launch_sgd(master, grad, counts, total, per_set, lr, lut, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ok() : cuda_fail(e, "SGD kernel launch");
 }
 
 sk_status sk_device_check(uint32_t* flags, int clear, sk_stream_t stream) {

@@ -347,6 +347,13 @@ cudaError_t launch_dlut_tc(const Problem& p, const uint16_t* X, const uint16_t* 
 size_t dlut_tc_workspace(int64_t n, int64_t d, int bits, int gpr);
 size_t dlut_noalloc_scratch_bytes();
 cudaError_t dlut_noalloc_scratch(void** ptr);
+cudaError_t launch_bin_counts(const uint8_t* packed, int64_t row_bytes, int bits, int64_t n, int gpr, int64_t gs,
+                              int32_t* counts, cudaStream_t s);
+cudaError_t launch_adamw(float* master, float* m, float* v, const float* grad, const int32_t* counts, int64_t total,
+                         int64_t per_set, float lr, float beta1, float beta2, float eps, float weight_decay, int step,
+                         uint16_t* lut, cudaStream_t s);
+cudaError_t launch_sgd(float* master, const float* grad, const int32_t* counts, int64_t total, int64_t per_set,
+                       float lr, uint16_t* lut, cudaStream_t s);
 cudaError_t launch_simt_bwd_input(const Problem& p, const uint16_t* dY, uint16_t* dX, cudaStream_t s);
 cudaError_t launch_simt_bwd_lut(const Problem& p, const uint16_t* X, const uint16_t* dY, float* dlut,
                                 int accumulate, cudaStream_t s);

@@ -23,7 +23,8 @@ SK_CHECK_INDEX_RANGE = 2
 EXPORTED = (
     "sk_abi_version", "sk_status_string", "sk_last_error", "sk_packed_row_bytes", "sk_packed_bytes",
     "sk_pack", "sk_unpack", "sk_dequant", "sk_workspace_bytes", "sk_linear_fwd", "sk_linear_bwd_input",
-    "sk_linear_bwd_lut", "sk_linear_bwd_lut_noalloc", "sk_device_check",
+    "sk_linear_bwd_lut", "sk_linear_bwd_lut_noalloc", "sk_bin_counts", "sk_lut_adamw", "sk_lut_sgd",
+    "sk_device_check",
 )
 
 
@@ -37,7 +38,7 @@ def _load() -> ctypes.CDLL:
     if not os.path.exists(_LIB_PATH):
         raise ImportError(f"{_LIB_PATH} is missing: build it with `python -m compressive_fine_tuning_b200.build`")
     lib = ctypes.CDLL(_LIB_PATH)
-    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    vp, i64, i32, sz, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
     sigs = {
         "sk_abi_version": ([], i32),
         "sk_status_string": ([i32], ctypes.c_char_p),
@@ -52,6 +53,9 @@ def _load() -> ctypes.CDLL:
         "sk_linear_bwd_input": ([vp, vp, i32, i32, i64, i64, vp, i64, vp, i32, vp, vp, sz, vp], i32),
         "sk_linear_bwd_lut": ([vp, i32, i32, i64, i64, vp, vp, i64, vp, i32, vp, i32, vp, sz, vp], i32),
         "sk_linear_bwd_lut_noalloc": ([vp, i32, i32, i64, i64, vp, vp, i64, vp, i32, vp, i32, vp], i32),
+        "sk_bin_counts": ([vp, i32, i32, i64, i64, vp, vp], i32),
+        "sk_lut_adamw": ([vp, vp, vp, vp, vp, i32, i64, i32, i32, f32, f32, f32, f32, f32, i32, vp, vp], i32),
+        "sk_lut_sgd": ([vp, vp, vp, i32, i64, i32, i32, f32, vp, vp], i32),
         "sk_device_check": ([ctypes.POINTER(ctypes.c_uint32), i32, vp], i32),
     }
     for name, (args, res) in sigs.items():
@@ -221,6 +225,47 @@ def device_check(clear: bool = True, device=None) -> int:
     if st not in (SK_OK, 4):
         _check(st)
     return int(flags.value)
+
+
+def bin_counts(packed: torch.Tensor, bits: int, gpr: int, n: int, d: int) -> torch.Tensor:
+    """Static bin sizes counts[i][g][c] of the index map (int32 [n, gpr, 2^bits])."""
+    _need(packed, torch.uint8, "packed")
+    out = torch.empty((n, gpr, 1 << bits), dtype=torch.int32, device=packed.device)
+    _check(lib.sk_bin_counts(_ptr(packed), bits, gpr, n, d, _ptr(out), _stream(packed.device)))
+    return out
+
+
+def _lut_update_shape(master: torch.Tensor, bits: int):
+    if master.dtype != torch.float32 or master.dim() != 4 or master.shape[-1] != (1 << bits) or not master.is_contiguous():
+        raise ValueError("master LUTs must be contiguous fp32 [ntask, n, gpr, 2^bits]")
+    return master.shape[0], master.shape[1], master.shape[2]
+
+
+def lut_adamw_(master: torch.Tensor, m: torch.Tensor, v: torch.Tensor, grad: torch.Tensor, bits: int, step: int,
+               lr: float, beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8, weight_decay: float = 0.0,
+               counts: Optional[torch.Tensor] = None, lut: Optional[torch.Tensor] = None) -> None:
+    """One AdamW step on fp32 master LUTs (in place); writes the fp16 LUTs when given.
+    counts (from bin_counts) selects the averaging variant of the gradient."""
+    ntask, n, gpr = _lut_update_shape(master, bits)
+    for t, name in ((m, "m"), (v, "v"), (grad, "grad")):
+        if t.shape != master.shape or t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError(f"{name} must match the master LUTs")
+    if lut is not None and (lut.shape != master.shape or lut.dtype != torch.float16 or not lut.is_contiguous()):
+        raise ValueError("lut must be contiguous fp16 of the master's shape")
+    _check(lib.sk_lut_adamw(_ptr(master), _ptr(m), _ptr(v), _ptr(grad), _ptr(counts), ntask, n, gpr, bits, lr, beta1,
+                            beta2, eps, weight_decay, step, _ptr(lut), _stream(master.device)))
+
+
+def lut_sgd_(master: torch.Tensor, grad: torch.Tensor, bits: int, lr: float, counts: Optional[torch.Tensor] = None,
+             lut: Optional[torch.Tensor] = None) -> None:
+    """One SGD step on fp32 master LUTs (in place); writes the fp16 LUTs when given."""
+    ntask, n, gpr = _lut_update_shape(master, bits)
+    if grad.shape != master.shape or grad.dtype != torch.float32 or not grad.is_contiguous():
+        raise ValueError("grad must match the master LUTs")
+    if lut is not None and (lut.shape != master.shape or lut.dtype != torch.float16 or not lut.is_contiguous()):
+        raise ValueError("lut must be contiguous fp16 of the master's shape")
+    _check(lib.sk_lut_sgd(_ptr(master), _ptr(grad), _ptr(counts), ntask, n, gpr, bits, lr, _ptr(lut),
+                          _stream(master.device)))
 
 
 class SketchedLinearFunction(torch.autograd.Function):

@@ -200,6 +200,43 @@ sk_status sk_linear_bwd_lut_noalloc(const void* packed, int bits, int gpr, int64
                                     sk_stream_t stream);
 
 /*
+ * sk_bin_counts: the static bin sizes of the one-hot sketch (Eq. 1),
+ * counts[i][g][c] = the number of columns j of group g in row i with
+ * idx[i][j] == c, as int32 [n][gpr][2^bits] in device memory.  They sum to
+ * d / gpr over c.  The averaging variant of the LUT update divides the LUT
+ * gradient by them (SpaLLM section 2.1: the gradients of the virtual
+ * parameters that share a trainable value are averaged).  Shape rules and
+ * errors as sk_linear_bwd_lut.
+ */
+sk_status sk_bin_counts(const void* packed, int bits, int gpr, int64_t n, int64_t d, int32_t* counts,
+                        sk_stream_t stream);
+
+/*
+ * sk_lut_adamw / sk_lut_sgd: one optimizer step on the LUT values.  The pages
+ * train the LUTs but name no optimizer; these are the plain textbook
+ * updates on fp32 master copies, elementwise over ntask * n * gpr * 2^bits
+ * entries (device fp32 arrays of that length, layout [ntask][n][gpr][k]):
+ *
+ *   g = grad / max(counts, 1)  if counts != NULL (averaging; counts [n][gpr][k]
+ *                               from sk_bin_counts, shared by every LUT set)
+ *   AdamW: p *= 1 - lr * weight_decay;  m = beta1 m + (1 - beta1) g;
+ *          v = beta2 v + (1 - beta2) g^2;
+ *          p -= lr * (m / (1 - beta1^step)) / (sqrt(v / (1 - beta2^step)) + eps)
+ *   SGD:   p -= lr * g
+ *
+ * master, m and v are updated in place (m and v start at zero); grad is the
+ * output of sk_linear_bwd_lut.  When lut is not NULL the fp16 LUTs the layer
+ * reads ([ntask][n][gpr][k], IEEE fp16 bits) receive the round-to-nearest-even
+ * fp16 of the new master values.  step >= 1; 0 <= beta1, beta2 < 1; eps > 0.
+ * Outputs must not overlap inputs other than themselves.
+ */
+sk_status sk_lut_adamw(float* master, float* m, float* v, const float* grad, const int32_t* counts, int ntask,
+                       int64_t n, int gpr, int bits, float lr, float beta1, float beta2, float eps,
+                       float weight_decay, int step, uint16_t* lut, sk_stream_t stream);
+sk_status sk_lut_sgd(float* master, const float* grad, const int32_t* counts, int ntask, int64_t n, int gpr,
+                     int bits, float lr, uint16_t* lut, sk_stream_t stream);
+
+/*
  * sk_device_check: synchronises `stream`, stores the device check word
  * (SK_CHECK_* bits, 0 = nothing flagged) in *flags and clears it if `clear`.
  * Returns SK_ERR_DEVICE_CHECK when any bit was set, else SK_OK.

@@ -9,7 +9,9 @@ Everything here is plain, slow and written to be checked by eye against the
 definitions on the pages: "SpaLLM: Unified Compressive Adaptation of LLMs with
 Sketching" (section 2.2, Eq. 1 and groups per row; section 2.3, multiple LUT
 sets; section 2.4, the identity example) and the "Sketch to Adapt" OpenReview
-discussion (the corrected Eq. 6 and the mapping matrix M).  Floating point is
+discussion (the corrected Eq. 6 and the mapping matrix M).  The LUT update
+(AdamW, SGD, the averaging of shared gradients of section 2.1) is the
+textbook optimizer the pages leave unnamed.  Floating point is
 float64 throughout; fp16 LUT values and bf16 activations widen exactly.
 
 Parity pins: every function here is pinned by a CPU test against something
@@ -20,5 +22,5 @@ from .sketch_oracle import (  # noqa: F401
     row_stride_bytes, packed_bytes, pack, unpack, dequant, sketch_matrix,
     dequant_via_sketch_matrix, forward, backward_input, backward_lut,
     eq6_forward, eq6_backward_lut, bin_counts, trainable_params, lora_params,
-    compression_factor,
+    compression_factor, averaged_gradient, adamw_step, sgd_step,
 )

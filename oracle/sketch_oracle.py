@@ -269,6 +269,43 @@ def bin_counts(idx: np.ndarray, gpr: int, k: int) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# LUT update (the pages train the LUT values but name no optimizer)
+# ---------------------------------------------------------------------------
+
+def averaged_gradient(grad: np.ndarray, counts: Optional[np.ndarray]) -> np.ndarray:
+    """The "averaging" variant of SpaLLM section 2.1: the gradient of a
+    trainable LUT entry divided by the number of virtual parameters that share
+    it (its static bin size; empty bins keep their zero gradient).  counts is
+    [n, gpr, k] and applies to every LUT set."""
+    grad = np.asarray(grad, dtype=np.float64)
+    if counts is None:
+        return grad
+    return grad / np.maximum(np.asarray(counts, dtype=np.float64), 1.0)
+
+
+def adamw_step(master: np.ndarray, m: np.ndarray, v: np.ndarray, grad: np.ndarray, step: int,
+               lr: float, beta1: float, beta2: float, eps: float, weight_decay: float,
+               counts: Optional[np.ndarray] = None):
+    """One AdamW step (Adam with decoupled weight decay), written out:
+    p <- p (1 - lr wd);  m <- b1 m + (1 - b1) g;  v <- b2 v + (1 - b2) g^2;
+    p <- p - lr (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps).
+    Returns the new (master, m, v) in float64."""
+    g = averaged_gradient(grad, counts)
+    p = np.asarray(master, dtype=np.float64) * (1.0 - lr * weight_decay)
+    m = beta1 * np.asarray(m, dtype=np.float64) + (1.0 - beta1) * g
+    v = beta2 * np.asarray(v, dtype=np.float64) + (1.0 - beta2) * g * g
+    mhat = m / (1.0 - beta1 ** step)
+    vhat = v / (1.0 - beta2 ** step)
+    p = p - lr * mhat / (np.sqrt(vhat) + eps)
+    return p, m, v
+
+
+def sgd_step(master: np.ndarray, grad: np.ndarray, lr: float, counts: Optional[np.ndarray] = None) -> np.ndarray:
+    """Plain gradient descent on the LUT values: p <- p - lr g."""
+    return np.asarray(master, dtype=np.float64) - lr * averaged_gradient(grad, counts)
+
+
+# ---------------------------------------------------------------------------
 # Counting identities used by the pages
 # ---------------------------------------------------------------------------
 

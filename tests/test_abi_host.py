@@ -130,3 +130,38 @@ def test_valid_call_without_device_fails_loudly():
     assert fwd() in (SK_ERR_CUDA, SK_ERR_UNSUPPORTED)
     assert bwd_in() in (SK_ERR_CUDA, SK_ERR_UNSUPPORTED)
     assert bwd_lut() in (SK_ERR_CUDA, SK_ERR_UNSUPPORTED)
+
+
+def _adamw(**kw):
+    a = dict(master=A, m=B, v=C, grad=ctypes.c_void_p(0x50000000), counts=None, ntask=1, n=8, gpr=2, bits=4,
+             lr=1e-3, b1=0.9, b2=0.999, eps=1e-8, wd=0.0, step=1, lut=ctypes.c_void_p(0x60000000))
+    a.update(kw)
+    return sk.lib.sk_lut_adamw(a["master"], a["m"], a["v"], a["grad"], a["counts"], a["ntask"], a["n"], a["gpr"],
+                               a["bits"], a["lr"], a["b1"], a["b2"], a["eps"], a["wd"], a["step"], a["lut"], None)
+
+
+def test_lut_update_validation():
+    assert _adamw(step=0) == SK_ERR_INVALID_ARG
+    assert _adamw(b1=1.0) == SK_ERR_INVALID_ARG
+    assert _adamw(b2=-0.1) == SK_ERR_INVALID_ARG
+    assert _adamw(eps=0.0) == SK_ERR_INVALID_ARG
+    assert _adamw(lr=float("nan")) == SK_ERR_INVALID_ARG
+    assert _adamw(bits=5) == SK_ERR_INVALID_ARG
+    assert _adamw(master=None) == SK_ERR_INVALID_ARG
+    assert _adamw(v=ctypes.c_void_p(0x20000004)) == SK_ERR_INVALID_ARG           # misaligned
+    assert _adamw(m=ctypes.c_void_p(0x10000000 + 64)) == SK_ERR_INVALID_ARG      # overlaps master
+    assert _adamw(lut=ctypes.c_void_p(0x50000000 + 16)) == SK_ERR_INVALID_ARG    # overlaps grad
+    L = sk.lib
+    assert L.sk_lut_sgd(A, None, None, 1, 8, 2, 4, 0.1, None, None) == SK_ERR_INVALID_ARG
+    assert L.sk_lut_sgd(A, B, None, 0, 8, 2, 4, 0.1, None, None) == SK_ERR_INVALID_ARG
+    assert L.sk_bin_counts(A, 4, 3, 8, 64, B, None) == SK_ERR_INVALID_ARG        # gpr does not divide d
+    assert L.sk_bin_counts(A, 4, 1, 8, 64, None, None) == SK_ERR_INVALID_ARG
+    assert L.sk_bin_counts(A, 4, 1, 8, 64, ctypes.c_void_p(0x10000000 + 32), None) == SK_ERR_INVALID_ARG  # overlap
+
+
+def test_lut_update_without_device_fails_loudly():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present")
+    assert _adamw() in (SK_ERR_CUDA, SK_ERR_UNSUPPORTED)
+    assert sk.lib.sk_lut_sgd(A, B, None, 1, 8, 2, 4, 0.1, None, None) in (SK_ERR_CUDA, SK_ERR_UNSUPPORTED)
