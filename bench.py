@@ -126,7 +126,7 @@ def kernel_name(op, T, w):
     """The library kernel a launch of this kind runs (the dispatch rules of sk_api.cu)."""
     if op == "fwd":
         if w["ntask"] > 1:
-            return "fwd_tc_kernel (routed)"
+            return "decode_kernel" if (T == 1 and w["bits"] == 4) else "fwd_tc_kernel (routed)"
         path = os.environ.get("SK_FWD_PATH", "")
         if w["bits"] == 4 and T <= 16 and path not in ("gemv", "tc"):
             return "decode_kernel"
@@ -142,7 +142,7 @@ def kernels_per_launch(op, T, w):
     """Library kernels one API call of this kind launches: the routed forward
     adds the routing and gather kernels, the tensor-core LUT gradient adds its
     reduction of partial bins."""
-    if op == "fwd" and w["ntask"] > 1:
+    if op == "fwd" and w["ntask"] > 1 and not (T == 1 and w["bits"] == 4):
         return 3
     if op == "dlut" and T >= 64:
         return 2

@@ -129,6 +129,15 @@ bool use_decode_fwd(const sk::Problem& p) {
 // Several LUT sets: the tensor-core forward needs the routing workspace.
 bool routed_fwd_possible(int64_t d, int ntask) { return ntask > 1 && ntask <= sk::kMaxRouteTasks && d >= 128; }
 
+// Several LUT sets in the input gradient: routed tensor-core dX under the same
+// rules as the single-set tensor-core backward (SK_BWD_PATH=simt|tc forces).
+bool routed_dx_possible(int64_t n, int64_t d, int64_t T, int ntask) {
+  if (ntask <= 1 || ntask > sk::kMaxRouteTasks || n < 64 || d < 64) return false;
+  const int forced = env_path("SK_BWD_PATH");
+  if (forced == 1) return false;
+  return forced == 2 || T >= kBwdTcMinT;
+}
+
 // Shape rules shared by the layer calls.
 sk_status check_shape(int bits, int gpr, int64_t n, int64_t d, int64_t T, int ntask) {
   if (bits < 2 || bits > 4) return fail(SK_ERR_INVALID_ARG, "bits must be 2, 3 or 4 (got %d)", bits);
@@ -250,6 +259,7 @@ size_t sk_workspace_bytes(int op, int64_t n, int64_t d, int bits, int gpr, int64
   if (op == SK_OP_BWD_LUT && use_tensor_cores_bwd(n, d, T, ntask))
     return sk::dlut_tc_workspace(n, d, bits, gpr);
   if (op == SK_OP_FWD && routed_fwd_possible(d, ntask)) return sk::fwd_tc_workspace(T, d, ntask);
+  if (op == SK_OP_BWD_INPUT && routed_dx_possible(n, d, T, ntask)) return sk::dx_tc_workspace(T, n, ntask);
   return 0;
 }
 
@@ -287,7 +297,10 @@ sk_status sk_linear_fwd(const void* packed, const uint16_t* lut, int bits, int g
   sk::Problem p = make_problem(packed, lut, bits, gpr, n, d, T, task, ntask, check);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (task != nullptr && routed_fwd_possible(d, ntask)) {
+  if (task != nullptr && ntask > 1 && use_decode_fwd(p)) {
+    // a single token: one LUT set, chosen on the device by the decode kernel
+    e = sk::launch_decode_fwd(p, X, Y, s);
+  } else if (task != nullptr && routed_fwd_possible(d, ntask)) {
     // several LUT sets: bucket the tokens by task and run the tensor-core
     // forward per task tile when the caller gave the routing workspace; without
     // it (or with SK_FWD_PATH=gemv) the CUDA-core kernel serves the batch
@@ -318,15 +331,23 @@ sk_status sk_linear_bwd_input(const void* packed, const uint16_t* lut, int bits,
   st = check_layer_buffers(packed, lut, true, bits, gpr, n, d, T, task, ntask, dY, (size_t)(T * n * 2), nullptr, 0, dX,
                            (size_t)(T * d * 2));
   if (st != SK_OK) return st;
-  if (workspace_bytes < sk_workspace_bytes(SK_OP_BWD_INPUT, n, d, bits, gpr, T, ntask))
-    return fail(SK_ERR_INVALID_ARG, "workspace too small");
   unsigned int* check = nullptr;
   st = device_state(&check);
   if (st != SK_OK) return st;
   sk::Problem p = make_problem(packed, lut, bits, gpr, n, d, T, task, ntask, check);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = use_tensor_cores_bwd(n, d, T, ntask) ? sk::launch_dx_tc(p, dY, dX, s)
-                                                                          : sk::launch_simt_bwd_input(p, dY, dX, s);
+  cudaError_t e;
+  if (task != nullptr && ntask > 1) {
+    // several LUT sets: tokens bucketed by task for the tensor cores when the
+    // caller gave the routing workspace, else the CUDA-core kernel
+    const size_t need = sk::dx_tc_workspace(T, n, ntask);
+    const bool ws_ok = workspace != nullptr && workspace_bytes >= need && aligned16(workspace) &&
+                       !overlaps(workspace, need, dY, (size_t)(T * n * 2)) && !overlaps(workspace, need, dX, (size_t)(T * d * 2));
+    e = (ws_ok && routed_dx_possible(n, d, T, ntask)) ? sk::launch_dx_tc_routed(p, dY, dX, workspace, s)
+                                                      : sk::launch_simt_bwd_input(p, dY, dX, s);
+  } else {
+    e = use_tensor_cores_bwd(n, d, T, ntask) ? sk::launch_dx_tc(p, dY, dX, s) : sk::launch_simt_bwd_input(p, dY, dX, s);
+  }
   return e == cudaSuccess ? ok() : cuda_fail(e, "input-gradient kernel launch");
 }
 

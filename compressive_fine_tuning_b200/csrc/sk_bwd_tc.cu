@@ -60,6 +60,12 @@ struct DxArgs {
   int gpr;
   uint16_t* dX;
   unsigned int* check;
+  // task-routed batches: dY rows are in task order, tile y covers positions
+  // [tiles[3y + 1], + tiles[3y + 2]) of task tiles[3y] and perm maps a
+  // position back to its token; nullptr for single-LUT-set batches
+  const int* tiles;
+  const int* perm;
+  int64_t lut_task_stride;
 };
 
 template <int BITS>
@@ -77,7 +83,19 @@ dx_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, DxArgs a) {
 
   const int warp = tc::warp_id(), lane = tc::lane_id();
   const int64_t j0 = (int64_t)blockIdx.x * 128;
-  const int t0 = blockIdx.y * N;
+  int t0 = blockIdx.y * N;            // first dY row of the tile
+  int64_t tlen = a.T - t0;            // tokens of the tile (bounded by N below)
+  const uint16_t* lut = a.lut;
+  if (a.tiles != nullptr) {
+    const int tau = a.tiles[3 * blockIdx.y];
+    t0 = a.tiles[3 * blockIdx.y + 1];
+    tlen = a.tiles[3 * blockIdx.y + 2];
+    if (tlen == 0) return;            // an unused tile: the whole CTA leaves before any setup
+    lut += (int64_t)tau * a.lut_task_stride;
+  }
+  if (tlen > N) tlen = N;
+  // output row of tile token t (positions map back to tokens when routed)
+  auto out_row = [&](int t) -> int64_t { return a.tiles != nullptr ? (int64_t)a.perm[t0 + t] : (int64_t)(t0 + t); };
   const int nsteps = ceil_div(a.n, KS);
 
   if (threadIdx.x == 0) {
@@ -151,7 +169,7 @@ dx_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, DxArgs a) {
       const int64_t row = (int64_t)i * KS + lr;
       if (col_ok && row < a.n) {
         ch_next = load_chunk<BITS>(a.packed + row * a.row_bytes, cchunk);
-        const uint16_t* lp = a.lut + (row * a.gpr + g) * (1 << BITS);
+        const uint16_t* lp = lut + (row * a.gpr + g) * (1 << BITS);
         if constexpr (BITS == 4) {
           lraw_next[0] = __ldg(reinterpret_cast<const uint4*>(lp));
           lraw_next[1] = __ldg(reinterpret_cast<const uint4*>(lp) + 1);
@@ -225,10 +243,10 @@ dx_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, DxArgs a) {
         if (j < a.d) {
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const int64_t t = t0 + gi * 16 + e;
-            if (t < a.T) {
+            const int t = gi * 16 + e;
+            if (t < tlen) {
               __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(v[e]));
-              a.dX[t * a.d + j] = *reinterpret_cast<uint16_t*>(&b);
+              a.dX[out_row(t) * a.d + j] = *reinterpret_cast<uint16_t*>(&b);
             }
           }
         }
@@ -439,13 +457,16 @@ size_t dlut_tc_workspace(int64_t n, int64_t d, int bits, int gpr) {
   return (size_t)jtiles * n * dlut_slots(gs, gpr) * (1 << bits) * sizeof(float);
 }
 
-cudaError_t launch_dx_tc(const Problem& p, const uint16_t* dY, uint16_t* dX, cudaStream_t s) {
+namespace {
+cudaError_t dx_launch(const Problem& p, const uint16_t* dY, uint16_t* dX, const Routed* rt, cudaStream_t s) {
   CUtensorMap tm;
-  cudaError_t e = make_tmap_2d(&tm, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)p.n, (uint64_t)p.T,
-                               (uint64_t)p.n * 2, 64, dx::N, CU_TENSOR_MAP_SWIZZLE_128B);
+  cudaError_t e = make_tmap_2d(&tm, rt != nullptr ? rt->Xp : dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)p.n,
+                               (uint64_t)p.T, (uint64_t)p.n * 2, 64, dx::N, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
-  DxArgs args{p.packed, p.row_bytes, p.lut, p.n, p.d, p.gs, p.T, p.gpr, dX, p.check};
-  dim3 grid((unsigned)ceil_div(p.d, 128), (unsigned)ceil_div(p.T, dx::N));
+  DxArgs args{p.packed, p.row_bytes, p.lut, p.n, p.d, p.gs, p.T, p.gpr, dX, p.check,
+              rt != nullptr ? rt->tiles : nullptr, rt != nullptr ? rt->perm : nullptr,
+              p.n * p.gpr * (1 << p.bits)};
+  dim3 grid((unsigned)ceil_div(p.d, 128), rt != nullptr ? (unsigned)rt->max_tiles : (unsigned)ceil_div(p.T, dx::N));
   auto run = [&](auto kern) {
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dx::SMEM);
     if (err != cudaSuccess) return err;
@@ -457,6 +478,20 @@ cudaError_t launch_dx_tc(const Problem& p, const uint16_t* dY, uint16_t* dX, cud
     case 3: return run(dx_tc_kernel<3>);
     default: return run(dx_tc_kernel<4>);
   }
+}
+}  // namespace
+
+cudaError_t launch_dx_tc(const Problem& p, const uint16_t* dY, uint16_t* dX, cudaStream_t s) {
+  return dx_launch(p, dY, dX, nullptr, s);
+}
+
+size_t dx_tc_workspace(int64_t T, int64_t n, int ntask) { return route_workspace_bytes(T, n, ntask, dx::N); }
+
+cudaError_t launch_dx_tc_routed(const Problem& p, const uint16_t* dY, uint16_t* dX, void* workspace, cudaStream_t s) {
+  Routed rt;
+  cudaError_t e = launch_route(p, dY, p.n, dX, p.d, dx::N, workspace, &rt, s);
+  if (e != cudaSuccess) return e;
+  return dx_launch(p, dY, dX, &rt, s);
 }
 
 cudaError_t launch_dlut_tc(const Problem& p, const uint16_t* X, const uint16_t* dY, float* dlut, int accumulate,

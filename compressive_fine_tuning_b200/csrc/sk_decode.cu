@@ -48,6 +48,10 @@ constexpr int kSmemBudget2 = 200 * 1024;          // two token tiles: one CTA pe
 
 struct DqArgs {
   const uint16_t* lut;
+  // a single token with a task id (several LUT sets): the LUT set is read on
+  // the device; nullptr when the batch has one LUT set
+  const int32_t* task;
+  int ntask;
   int64_t n, d, gs;
   int gpr, T;
   int tiles;          // ceil(n / 16)
@@ -176,12 +180,25 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constant__
     uint8_t* planes = smem + a.lut_off;
     const int tid = threadIdx.x < kDqWarps * 32 ? threadIdx.x : threadIdx.x - 1;   // skip the producer thread
     const int nthr = kDqThreads - 1;
+    const uint16_t* lut = a.lut;
+    if (a.task != nullptr) {
+      // the token's LUT set: task ids are inputs, so read them after the wait;
+      // an id outside [0, ntask) gets all-zero LUTs (a zero output row) and a flag
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      const int tau = __ldg(a.task);
+      if (tau < 0 || tau >= a.ntask) {
+        lut = nullptr;
+        if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(a.check, SK_CHECK_TASK_RANGE);
+      } else {
+        lut += (int64_t)tau * a.n * gpr * 16;
+      }
+    }
     for (int e = tid; e < RT * kTileRows * gpr; e += nthr) {
       const int r = e / gpr, g = e - r * gpr;
       uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
-      if (row0 + r < a.n) {
+      if (row0 + r < a.n && lut != nullptr) {
         LutRegs<4> L;
-        load_lut<4>(a.lut + ((row0 + r) * gpr + g) * 16, L);
+        load_lut<4>(lut + ((row0 + r) * gpr + g) * 16, L);
         lo = make_uint4(L.lo[0], L.lo[1], L.lo[2], L.lo[3]);
         hi = make_uint4(L.hi[0], L.hi[1], L.hi[2], L.hi[3]);
       }
@@ -464,7 +481,8 @@ __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / 
 bool plan(const Problem& p, DqArgs* a, int* grid, int* smem, int* seg) {
   // d % 256 == 0: index rows are whole 128-byte blocks (the 3-D box never
   // reaches past a row), X rows whole 256-column blocks
-  if (p.bits != 4 || p.T < 1 || p.T > 16 || p.d % kBoxCols != 0 || (p.task != nullptr && p.ntask != 1)) return false;
+  if (p.bits != 4 || p.T < 1 || p.T > 16 || p.d % kBoxCols != 0) return false;
+  if (p.task != nullptr && p.ntask != 1 && p.T != 1) return false;   // several LUT sets: one token only
   const int tiles = (int)((p.n + kTileRows - 1) / kTileRows);
   const int sms = num_sms();
   int G = tiles < sms ? tiles : sms;
@@ -492,7 +510,8 @@ bool plan(const Problem& p, DqArgs* a, int* grid, int* smem, int* seg) {
     const int total = 1024 + S * stage + lut_bytes + red_bytes + bar_bytes;
     if (total > budget && SEG > 512) continue;
     if (total > 227 * 1024) return false;
-    a->lut = p.lut; a->n = p.n; a->d = p.d; a->gs = p.gs; a->gpr = p.gpr; a->T = T;
+    a->lut = p.lut; a->task = (p.task != nullptr && p.ntask != 1) ? p.task : nullptr; a->ntask = p.ntask;
+    a->n = p.n; a->d = p.d; a->gs = p.gs; a->gpr = p.gpr; a->T = T;
     a->tiles = tiles; a->segs = segs; a->stages = S; a->rt_max = rt_max;
     a->stage_bytes = stage; a->x_off = idx_region;
     a->lut_off = S * stage; a->lut_pitch = lut_pitch;

@@ -419,7 +419,7 @@ template <int BITS>
 cudaError_t launch_bits_routed(const Problem& p, const uint16_t* X, uint16_t* Y, void* ws, cudaStream_t s) {
   const int N = fwd_tc_tile_n(p.T, p.ntask);
   Routed rt;
-  cudaError_t e = launch_route(p, X, Y, N, ws, &rt, s);
+  cudaError_t e = launch_route(p, X, p.d, Y, p.n, N, ws, &rt, s);
   if (e != cudaSuccess) return e;
   switch (N) {
     case 16: return launch_n<BITS, 16>(p, X, Y, s, &rt);

@@ -317,8 +317,11 @@ struct Routed {
 };
 int route_max_tiles(int64_t T, int ntask, int N);
 size_t route_workspace_bytes(int64_t T, int64_t d, int ntask, int N);
-cudaError_t launch_route(const Problem& p, const uint16_t* X, uint16_t* Y, int N, void* workspace, Routed* out,
-                         cudaStream_t s);
+// Routes the tokens by task (tiles of at most N tokens) and gathers the rows
+// of `src` (src_width bf16 each) into task order; out_rows (out_width each)
+// gets zero rows for tokens with an out-of-range task id.
+cudaError_t launch_route(const Problem& p, const uint16_t* src, int64_t src_width, uint16_t* out_rows,
+                         int64_t out_width, int N, void* workspace, Routed* out, cudaStream_t s);
 // Token tile of the tensor-core forward for a batch of T tokens spread over
 // ntask LUT sets (16 ... 256).
 int fwd_tc_tile_n(int64_t T, int ntask);
@@ -342,6 +345,10 @@ bool decode_fwd_supported(const Problem& p);
 cudaError_t launch_decode_fwd(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStream_t s);
 cudaError_t launch_fwd_tc(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStream_t s);
 cudaError_t launch_dx_tc(const Problem& p, const uint16_t* dY, uint16_t* dX, cudaStream_t s);
+// dX for a batch with several LUT sets: tokens routed by task (workspace of
+// dx_tc_workspace bytes), one LUT set per 256-token tile.
+size_t dx_tc_workspace(int64_t T, int64_t n, int ntask);
+cudaError_t launch_dx_tc_routed(const Problem& p, const uint16_t* dY, uint16_t* dX, void* workspace, cudaStream_t s);
 cudaError_t launch_dlut_tc(const Problem& p, const uint16_t* X, const uint16_t* dY, float* dlut, int accumulate,
                            void* workspace, cudaStream_t s);
 size_t dlut_tc_workspace(int64_t n, int64_t d, int bits, int gpr);

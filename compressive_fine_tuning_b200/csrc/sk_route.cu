@@ -1,4 +1,4 @@
-// Task routing for the tensor-core forward ("SpaLLM: Unified Compressive
+// Task routing for the tensor-core kernels ("SpaLLM: Unified Compressive
 // Adaptation of LLMs with Sketching", section 2.3: several LUT sets share one
 // index map; every token uses its own task's set).
 //
@@ -9,8 +9,9 @@
 //     and the tile list (task, first position, length) with at most N tokens
 //     per tile; tokens with an out-of-range task id are left out, flagged in
 //     the check word and get a zero output row;
-//   * gather_kernel copies X's rows into segment order.
-// The forward kernel then runs over the tiles and scatters each output row
+//   * gather_kernel copies the input rows (X for the forward, dY for the input
+//     gradient) into segment order.
+// The product kernel then runs over the tiles and scatters each output row
 // back to its token.  A token's output does not depend on which other tokens
 // share its tile, so the order inside a segment does not matter.
 #include "sk_internal.cuh"
@@ -87,21 +88,21 @@ size_t route_workspace_bytes(int64_t T, int64_t d, int ntask, int N) {
   return head + (size_t)T * d * 2;
 }
 
-cudaError_t launch_route(const Problem& p, const uint16_t* X, uint16_t* Y, int N, void* workspace, Routed* out,
-                         cudaStream_t s) {
+cudaError_t launch_route(const Problem& p, const uint16_t* src, int64_t src_width, uint16_t* out_rows,
+                         int64_t out_width, int N, void* workspace, Routed* out, cudaStream_t s) {
   const int max_tiles = route_max_tiles(p.T, p.ntask, N);
   int* perm = static_cast<int*>(workspace);
   int* tiles = perm + p.T;
   int* valid = tiles + 3 * max_tiles;
   const size_t words = (size_t)p.T + 3 * (size_t)max_tiles + 1;
   uint16_t* Xp = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) + (words * 4 + 255) / 256 * 256);
-  route_kernel<<<1, kRouteThreads, 0, s>>>(p.task, (int)p.T, p.ntask, N, perm, tiles, max_tiles, valid, Y, p.n,
-                                           p.check);
+  route_kernel<<<1, kRouteThreads, 0, s>>>(p.task, (int)p.T, p.ntask, N, perm, tiles, max_tiles, valid, out_rows,
+                                           out_width, p.check);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int64_t units = p.d / 8;
+  const int64_t units = src_width / 8;
   const int64_t total = p.T * units;
-  gather_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(reinterpret_cast<const uint4*>(X), perm, valid,
+  gather_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(reinterpret_cast<const uint4*>(src), perm, valid,
                                                                 (int)p.T, units, reinterpret_cast<uint4*>(Xp));
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

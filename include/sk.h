@@ -126,6 +126,8 @@ sk_status sk_dequant(const void* packed, const uint16_t* lut, int bits, int gpr,
  * SK_OP_FWD with ntask > 1: the task routing of the tensor-core forward
  * (permutation, tile list and X in task order); optional -- without it a
  * batch with several LUT sets runs on the CUDA-core kernel.
+ * SK_OP_BWD_INPUT with ntask > 1: the same routing for the tensor-core input
+ * gradient (dY in task order); optional in the same way.
  */
 size_t sk_workspace_bytes(int op, int64_t n, int64_t d, int bits, int gpr,
                           int64_t T, int ntask);

@@ -97,3 +97,28 @@ def test_decode_identity_is_exact(monkeypatch):
     X = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
     Y = sk.linear_fwd(packed, torch.from_numpy(lut).cuda(), 4, X, None)
     np.testing.assert_array_equal(Y.view(torch.int16).cpu().numpy().view(np.uint16), x)
+
+
+@pytest.mark.parametrize("tau", [0, 5, 7])
+def test_decode_single_token_multitask(tau):
+    """One token with a task id picks its LUT set on the device (SpaLLM section
+    2.3); the routed path is not needed for a single token."""
+    from compressive_fine_tuning_b200 import sk
+    c = synth.layer_case(35000 + tau, n=1024, d=2048, bits=4, gpr=4, T=1, ntask=8, with_task=True)
+    c.task[:] = tau
+    packed, lut, X, dY, task = gc.dev_case(c)
+    sk.device_check(clear=True)
+    Y = sk.linear_fwd(packed, lut, 4, X, task)
+    gc.check_fwd(c, Y)
+    assert sk.device_check() == 0
+
+
+def test_decode_single_token_bad_task_zeroes_and_flags():
+    from compressive_fine_tuning_b200 import sk
+    c = synth.layer_case(35100, n=512, d=1024, bits=4, gpr=2, T=1, ntask=4, with_task=True)
+    packed, lut, X, dY, task = gc.dev_case(c)
+    task.fill_(9)
+    sk.device_check(clear=True)
+    Y = sk.linear_fwd(packed, lut, 4, X, task)
+    assert sk.device_check(clear=True) & sk.SK_CHECK_TASK_RANGE
+    assert not Y.float().abs().any()

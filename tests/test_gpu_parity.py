@@ -367,3 +367,48 @@ def test_multitask_forward_skewed_tasks():
     packed, lut, X, dY, task = gc.dev_case(c)
     gc.check_fwd(c, sk.linear_fwd(packed, lut, c.bits, X, task))
     assert sk.device_check() == 0
+
+
+# ---------------------------------------------------------------------------
+# several LUT sets on the tensor-core input gradient (task routing)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("path", ["auto", "simt", "tc"])
+@pytest.mark.parametrize("T,ntask,shape", [(64, 8, (136, 512, 3, 2)), (300, 3, (264, 1376, 2, 1)),
+                                           (1000, 8, (256, 1024, 4, 4)), (513, 2, (512, 2048, 4, 4)),
+                                           (17, 4, (128, 256, 4, 1))])
+def test_multitask_input_gradient_each_path(monkeypatch, path, T, ntask, shape):
+    sk = _sk()
+    if path != "auto":
+        monkeypatch.setenv("SK_BWD_PATH", path)
+    n, d, bits, gpr = shape
+    c = synth.layer_case(9900 + T, n=n, d=d, bits=bits, gpr=gpr, T=T, ntask=ntask)
+    packed, lut, X, dY, task = gc.dev_case(c)
+    if path == "tc" or (path == "auto" and T >= 64):
+        assert sk.workspace_bytes(sk.SK_OP_BWD_INPUT, n, d, bits, gpr, T, ntask) > 0
+    gc.check_bwd_input(c, sk.linear_bwd_input(packed, lut, c.bits, c.d, dY, task))
+    assert sk.device_check() == 0
+
+
+def test_multitask_input_gradient_skewed_and_bad_tasks(monkeypatch):
+    """Most tokens on one task, one task empty, two tokens with task ids out of
+    range: their dX rows are zero and the check word is flagged."""
+    sk = _sk()
+    c = synth.layer_case(9950, n=256, d=1024, bits=4, gpr=4, T=700, ntask=5)
+    c.task[:] = 0
+    c.task[::97] = 2
+    c.task[5] = 4
+    packed, lut, X, dY, task = gc.dev_case(c)
+    gc.check_bwd_input(c, sk.linear_bwd_input(packed, lut, c.bits, c.d, dY, task))
+    assert sk.device_check() == 0
+    task[3] = 9
+    task[400] = -1
+    sk.device_check(clear=True)
+    dX = sk.linear_bwd_input(packed, lut, c.bits, c.d, dY, task)
+    assert sk.device_check(clear=True) & sk.SK_CHECK_TASK_RANGE
+    assert not dX[3].float().abs().any() and not dX[400].float().abs().any()
+    keep = np.ones(c.T, dtype=bool)
+    keep[[3, 400]] = False
+    ref = oracle.backward_input(c.dy[keep], c.idx, c.lut, c.task[keep])
+    bound = oracle.backward_input(np.abs(c.dy[keep]), c.idx, np.abs(c.lut.astype(np.float64)), c.task[keep])
+    gc.check_rows(gc.bf16_to_f64(dX)[keep], ref, bound, "dX")
