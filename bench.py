@@ -52,6 +52,8 @@ WORKLOADS = {
                      desc="LLaMA-2-7B-shaped decode, 7 layers, 4-bit, GPR=8, T=1 and T=16"),
     "finetune7b": dict(shapes="LLAMA2_7B", bits=2, gpr=8, batches=(8192,), ntask=1, ops=("fwd", "dx", "dlut"),
                        desc="7B-shaped fine-tune step, 7 layers, 2-bit, GPR=8, T=8192: Y, dX, dLUT"),
+    "finetune7b_mt": dict(shapes="LLAMA2_7B", bits=2, gpr=8, batches=(8192,), ntask=8, ops=("fwd", "dx", "dlut"),
+                          desc="7B-shaped multi-task fine-tune step, 7 layers, 2-bit, GPR=8, 8 LUT sets, T=8192: Y, dX, dLUT"),
     "train13b": dict(shapes="LLAMA2_13B", bits=3, gpr=1, batches=(4096,), ntask=1, ops=("fwd", "dx", "dlut"),
                      desc="LLaMA-2-13B-shaped fwd+bwd, 7 layers, 3-bit, GPR=1, T=4096"),
     "serve70b_decode": dict(shapes="LLAMA3_70B", bits=4, gpr=4, batches=(1, 64), ntask=8, ops=("fwd",),
@@ -133,9 +135,10 @@ def kernel_name(op, T, w):
         if path == "gemv" or (T == 1 and path != "tc"):
             return "gemv_fwd_single_kernel"
         return "fwd_tc_kernel"
+    routed = " (routed)" if w["ntask"] > 1 else ""
     if op == "dx":
-        return "dx_tc_kernel" if T >= 64 else "simt_bwd_input_kernel"
-    return "dlut_tc_kernel" if T >= 64 else "simt_bwd_lut_kernel"
+        return "dx_tc_kernel" + routed if T >= 64 else "simt_bwd_input_kernel"
+    return "dlut_tc_kernel" + routed if T >= 64 else "simt_bwd_lut_kernel"
 
 
 def kernels_per_launch(op, T, w):
@@ -143,9 +146,11 @@ def kernels_per_launch(op, T, w):
     adds the routing and gather kernels, the tensor-core LUT gradient adds its
     reduction of partial bins."""
     if op == "fwd" and w["ntask"] > 1 and not (T == 1 and w["bits"] == 4):
-        return 3
+        return 3                    # route, gather, forward
+    if op == "dx" and w["ntask"] > 1 and T >= 64:
+        return 3                    # route, gather, input gradient
     if op == "dlut" and T >= 64:
-        return 2
+        return 5 if w["ntask"] > 1 else 2   # (route, two gathers,) bins, reduction
     return 1
 
 
@@ -247,7 +252,7 @@ def cpu_baseline(w, budget_s=15.0, seed=0):
             if "dx" in w["ops"]:
                 oracle.backward_input(c.dy, c.idx, c.lut, c.task)
             if "dlut" in w["ops"]:
-                oracle.backward_lut(c.x, c.dy, c.idx, gpr, 1 << bits)
+                oracle.backward_lut(c.x, c.dy, c.idx, gpr, 1 << bits, task=c.task, ntask=w["ntask"])
             dt = time.perf_counter() - s0
             if is_hbm_bound(w):
                 present = min(w["ntask"], Ts)

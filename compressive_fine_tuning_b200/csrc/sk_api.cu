@@ -260,6 +260,8 @@ size_t sk_workspace_bytes(int op, int64_t n, int64_t d, int bits, int gpr, int64
     return sk::dlut_tc_workspace(n, d, bits, gpr);
   if (op == SK_OP_FWD && routed_fwd_possible(d, ntask)) return sk::fwd_tc_workspace(T, d, ntask);
   if (op == SK_OP_BWD_INPUT && routed_dx_possible(n, d, T, ntask)) return sk::dx_tc_workspace(T, n, ntask);
+  if (op == SK_OP_BWD_LUT && routed_dx_possible(n, d, T, ntask))
+    return sk::dlut_tc_routed_workspace(n, d, bits, gpr, T, ntask);
   return 0;
 }
 
@@ -370,7 +372,8 @@ sk_status sk_linear_bwd_lut(const void* packed, int bits, int gpr, int64_t n, in
   st = check_layer_buffers(packed, nullptr, false, bits, gpr, n, d, T, task, ntask, X, (size_t)(T * d * 2), dY,
                            (size_t)(T * n * 2), dlut, dlut_bytes);
   if (st != SK_OK) return st;
-  if (workspace_bytes < sk_workspace_bytes(SK_OP_BWD_LUT, n, d, bits, gpr, T, ntask))
+  const bool routed = task != nullptr && ntask > 1;
+  if (!routed && workspace_bytes < sk_workspace_bytes(SK_OP_BWD_LUT, n, d, bits, gpr, T, ntask))
     return fail(SK_ERR_INVALID_ARG, "workspace too small");
   unsigned int* check = nullptr;
   st = device_state(&check);
@@ -378,7 +381,17 @@ sk_status sk_linear_bwd_lut(const void* packed, int bits, int gpr, int64_t n, in
   sk::Problem p = make_problem(packed, nullptr, bits, gpr, n, d, T, task, ntask, check);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (use_tensor_cores_bwd(n, d, T, ntask)) {
+  if (routed) {
+    // several LUT sets: the tokens of every set form their own K range of the
+    // tensor-core product when the caller gave the routing workspace, else
+    // the CUDA-core kernel
+    const size_t need = sk::dlut_tc_routed_workspace(n, d, bits, gpr, T, ntask);
+    const bool ws_ok = workspace != nullptr && workspace_bytes >= need && aligned16(workspace) &&
+                       !overlaps(workspace, need, X, (size_t)(T * d * 2)) && !overlaps(workspace, need, dY, (size_t)(T * n * 2)) &&
+                       !overlaps(workspace, need, dlut, dlut_bytes);
+    e = (ws_ok && routed_dx_possible(n, d, T, ntask)) ? sk::launch_dlut_tc_routed(p, X, dY, dlut, accumulate, workspace, s)
+                                                      : sk::launch_simt_bwd_lut(p, X, dY, dlut, accumulate, s);
+  } else if (use_tensor_cores_bwd(n, d, T, ntask)) {
     const size_t need = sk::dlut_tc_workspace(n, d, bits, gpr);
     if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))
       return fail(SK_ERR_INVALID_ARG, "workspace of %zu bytes (16-byte aligned) required", need);

@@ -291,8 +291,13 @@ struct DlutArgs {
   int64_t row_bytes;
   int64_t n, d, gs, T;
   int gpr, slots;
-  float* part;          // [jtiles][n][slots][k] partial bins
+  float* part;          // [jtiles][n][slots][k] partial bins (per LUT set when routed)
   unsigned int* check;
+  // several LUT sets: X and dY rows in task order, task z's tokens at
+  // positions [segs[2z], segs[2z] + segs[2z + 1]) (64-aligned, zero-padded);
+  // nullptr for one LUT set
+  const int* segs;
+  int64_t part_task_stride;  // floats between the partial bins of consecutive LUT sets
 };
 
 template <int BITS>
@@ -312,7 +317,14 @@ dlut_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant_
   const int jt = blockIdx.x;
   const int64_t j0 = (int64_t)jt * N;
   const int64_t i0 = (int64_t)blockIdx.y * M;
-  const int nsteps = ceil_div(a.T, KS);
+  int k_first = 0;                    // first token position of this LUT set
+  int nsteps = ceil_div(a.T, KS);
+  float* part = a.part;
+  if (a.segs != nullptr) {
+    k_first = a.segs[2 * blockIdx.z];
+    nsteps = ceil_div(a.segs[2 * blockIdx.z + 1], KS);   // a set with no tokens writes zero partials
+    part += (int64_t)blockIdx.z * a.part_task_stride;
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -341,7 +353,7 @@ dlut_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant_
         if (!tc::mbar_wait(&empty[s], ((i / S) & 1) ^ 1, a.check)) { *abort_flag = 1; break; }
         uint8_t* st = smem + s * STAGE;
         tc::mbar_arrive_expect_tx(&full[s], STAGE);
-        const int tk = i * KS;
+        const int tk = k_first + i * KS;
         tc::tma_load_2d(st, &tm_dy, &full[s], (int)i0, tk);
         tc::tma_load_2d(st + 8192, &tm_dy, &full[s], (int)i0 + 64, tk);
 #pragma unroll
@@ -373,7 +385,7 @@ dlut_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant_
     float* bins = reinterpret_cast<float*>(smem + BAR_OFF - K * 128 * 4);  // [K][128], tail of stage memory
     const int tid = threadIdx.x;                                         // 0..127
     const int64_t i = i0 + tid;
-    bool have = !*abort_flag && tc::mbar_wait(d_full, 0, a.check);
+    bool have = !*abort_flag && tc::mbar_wait(d_full, 0, a.check) && nsteps > 0;   // no steps: nothing accumulated
     have = __all_sync(0xffffffffu, have);  // tcgen05.ld is warp-collective
     if (have) tc::tc_fence_after();
     // the bins reuse the last stage's memory: wait until every MMA has read it (d_full)
@@ -385,7 +397,7 @@ dlut_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant_
     bool dirty = false;
     auto flush = [&](int gg) {
       if (i < a.n) {
-        float* dst = a.part + (((int64_t)jt * a.n + i) * a.slots + (gg - first_g)) * K;
+        float* dst = part + (((int64_t)jt * a.n + i) * a.slots + (gg - first_g)) * K;
 #pragma unroll
         for (int c = 0; c < K; ++c) dst[c] = bins[c * 128 + tid];
       }
@@ -430,12 +442,17 @@ dlut_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant_
 // the group, in tile order, and write (or add to) dlut.
 template <int BITS>
 __global__ void dlut_reduce_kernel(const float* __restrict__ part, int64_t n, int gpr, int64_t gs, int jtiles,
-                                   int slots, float* __restrict__ dlut, int accumulate) {
+                                   int slots, float* __restrict__ dlut, int accumulate, int ntask,
+                                   int64_t part_task_stride) {
   constexpr int K = 1 << BITS;
   const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= n * gpr * K) return;
-  const int c = (int)(e % K);
-  const int64_t ig = e / K;
+  const int64_t per_set = n * gpr * K;
+  if (e >= per_set * ntask) return;
+  const int64_t tau = e / per_set;
+  part += tau * part_task_stride;
+  const int64_t es = e - tau * per_set;
+  const int c = (int)(es % K);
+  const int64_t ig = es / K;
   const int g = (int)(ig % gpr);
   const int64_t i = ig / gpr;
   const int t_first = (int)(((int64_t)g * gs) / dl::N);
@@ -494,20 +511,26 @@ cudaError_t launch_dx_tc_routed(const Problem& p, const uint16_t* dY, uint16_t* 
   return dx_launch(p, dY, dX, &rt, s);
 }
 
-cudaError_t launch_dlut_tc(const Problem& p, const uint16_t* X, const uint16_t* dY, float* dlut, int accumulate,
-                           void* workspace, cudaStream_t s) {
+namespace {
+// part: partial bins; rp: the padded task routing (nullptr for one LUT set)
+cudaError_t dlut_launch(const Problem& p, const uint16_t* X, const uint16_t* dY, float* dlut, int accumulate,
+                        float* part, const RoutedPad* rp, cudaStream_t s) {
+  const uint64_t rows = rp != nullptr ? (uint64_t)rp->positions : (uint64_t)p.T;
   CUtensorMap tm_dy, tm_x;
-  cudaError_t e = make_tmap_2d(&tm_dy, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)p.n, (uint64_t)p.T,
-                               (uint64_t)p.n * 2, 64, dl::KS, CU_TENSOR_MAP_SWIZZLE_128B);
+  cudaError_t e = make_tmap_2d(&tm_dy, rp != nullptr ? rp->b : dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)p.n,
+                               rows, (uint64_t)p.n * 2, 64, dl::KS, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
-  e = make_tmap_2d(&tm_x, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)p.d, (uint64_t)p.T, (uint64_t)p.d * 2,
-                   64, dl::KS, CU_TENSOR_MAP_SWIZZLE_128B);
+  e = make_tmap_2d(&tm_x, rp != nullptr ? rp->a : X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)p.d, rows,
+                   (uint64_t)p.d * 2, 64, dl::KS, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
   const int slots = dlut_slots(p.gs, p.gpr);
   const int jtiles = ceil_div(p.d, dl::N);
-  DlutArgs args{p.packed, p.row_bytes, p.n, p.d, p.gs, p.T, p.gpr, slots, static_cast<float*>(workspace), p.check};
-  dim3 grid((unsigned)jtiles, (unsigned)ceil_div(p.n, dl::M));
-  const int64_t outs = p.n * p.gpr * (1 << p.bits);
+  const int sets = rp != nullptr ? p.ntask : 1;
+  const int64_t stride = (int64_t)jtiles * p.n * slots * (1 << p.bits);
+  DlutArgs args{p.packed, p.row_bytes, p.n, p.d, p.gs, p.T, p.gpr, slots, part, p.check,
+                rp != nullptr ? rp->segs : nullptr, stride};
+  dim3 grid((unsigned)jtiles, (unsigned)ceil_div(p.n, dl::M), (unsigned)sets);
+  const int64_t outs = (int64_t)sets * p.n * p.gpr * (1 << p.bits);
   const unsigned rgrid = (unsigned)((outs + 255) / 256);
   auto run = [&](auto kern, auto red) {
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dl::SMEM);
@@ -515,7 +538,7 @@ cudaError_t launch_dlut_tc(const Problem& p, const uint16_t* X, const uint16_t* 
     kern<<<grid, dl::THREADS, dl::SMEM, s>>>(tm_dy, tm_x, args);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
-    red<<<rgrid, 256, 0, s>>>(static_cast<const float*>(workspace), p.n, p.gpr, p.gs, jtiles, slots, dlut, accumulate);
+    red<<<rgrid, 256, 0, s>>>(part, p.n, p.gpr, p.gs, jtiles, slots, dlut, accumulate, sets, stride);
     return cudaGetLastError();
   };
   switch (p.bits) {
@@ -523,6 +546,29 @@ cudaError_t launch_dlut_tc(const Problem& p, const uint16_t* X, const uint16_t* 
     case 3: return run(dlut_tc_kernel<3>, dlut_reduce_kernel<3>);
     default: return run(dlut_tc_kernel<4>, dlut_reduce_kernel<4>);
   }
+}
+}  // namespace
+
+cudaError_t launch_dlut_tc(const Problem& p, const uint16_t* X, const uint16_t* dY, float* dlut, int accumulate,
+                           void* workspace, cudaStream_t s) {
+  return dlut_launch(p, X, dY, dlut, accumulate, static_cast<float*>(workspace), nullptr, s);
+}
+
+// workspace: the padded routing (positions, segments, X and dY in task order),
+// then the partial bins of every LUT set
+size_t dlut_tc_routed_workspace(int64_t n, int64_t d, int bits, int gpr, int64_t T, int ntask) {
+  const size_t route = route_pad_workspace_bytes(T, d, n, ntask, dl::KS);
+  return (route + 255) / 256 * 256 + (size_t)ntask * dlut_tc_workspace(n, d, bits, gpr);
+}
+
+cudaError_t launch_dlut_tc_routed(const Problem& p, const uint16_t* X, const uint16_t* dY, float* dlut, int accumulate,
+                                  void* workspace, cudaStream_t s) {
+  RoutedPad rp;
+  cudaError_t e = launch_route_padded(p, X, p.d, dY, p.n, dl::KS, workspace, &rp, s);
+  if (e != cudaSuccess) return e;
+  const size_t route = route_pad_workspace_bytes(p.T, p.d, p.n, p.ntask, dl::KS);
+  float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + (route + 255) / 256 * 256);
+  return dlut_launch(p, X, dY, dlut, accumulate, part, &rp, s);
 }
 
 }  // namespace sk

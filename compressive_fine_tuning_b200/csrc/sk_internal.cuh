@@ -322,6 +322,18 @@ size_t route_workspace_bytes(int64_t T, int64_t d, int ntask, int N);
 // gets zero rows for tokens with an out-of-range task id.
 cudaError_t launch_route(const Problem& p, const uint16_t* src, int64_t src_width, uint16_t* out_rows,
                          int64_t out_width, int N, void* workspace, Routed* out, cudaStream_t s);
+// Padded routing for the LUT gradient: task segments start at multiples of
+// `pad` positions (empty positions hold zero rows); two inputs gathered.
+struct RoutedPad {
+  const int* segs;     // [ntask][2]: first position, token count
+  int positions;       // rows of the gathered inputs
+  const uint16_t* a;   // [positions][width_a]
+  const uint16_t* b;   // [positions][width_b]
+};
+int route_pad_positions(int64_t T, int ntask, int pad);
+size_t route_pad_workspace_bytes(int64_t T, int64_t width_a, int64_t width_b, int ntask, int pad);
+cudaError_t launch_route_padded(const Problem& p, const uint16_t* a, int64_t width_a, const uint16_t* b,
+                                int64_t width_b, int pad, void* workspace, RoutedPad* out, cudaStream_t s);
 // Token tile of the tensor-core forward for a batch of T tokens spread over
 // ntask LUT sets (16 ... 256).
 int fwd_tc_tile_n(int64_t T, int ntask);
@@ -352,6 +364,11 @@ cudaError_t launch_dx_tc_routed(const Problem& p, const uint16_t* dY, uint16_t* 
 cudaError_t launch_dlut_tc(const Problem& p, const uint16_t* X, const uint16_t* dY, float* dlut, int accumulate,
                            void* workspace, cudaStream_t s);
 size_t dlut_tc_workspace(int64_t n, int64_t d, int bits, int gpr);
+// LUT gradient for a batch with several LUT sets: tokens routed by task into
+// 64-token-aligned segments, one K range per task.
+size_t dlut_tc_routed_workspace(int64_t n, int64_t d, int bits, int gpr, int64_t T, int ntask);
+cudaError_t launch_dlut_tc_routed(const Problem& p, const uint16_t* X, const uint16_t* dY, float* dlut, int accumulate,
+                                  void* workspace, cudaStream_t s);
 size_t dlut_noalloc_scratch_bytes();
 cudaError_t dlut_noalloc_scratch(void** ptr);
 cudaError_t launch_bin_counts(const uint8_t* packed, int64_t row_bytes, int bits, int64_t n, int gpr, int64_t gs,

@@ -128,6 +128,11 @@ sk_status sk_dequant(const void* packed, const uint16_t* lut, int bits, int gpr,
  * batch with several LUT sets runs on the CUDA-core kernel.
  * SK_OP_BWD_INPUT with ntask > 1: the same routing for the tensor-core input
  * gradient (dY in task order); optional in the same way.
+ * SK_OP_BWD_LUT with ntask > 1 (and task ids): the task routing of the
+ * tensor-core LUT gradient (X and dY in task order, each set's tokens padded
+ * to a multiple of 64 positions) plus the partial bins of every LUT set;
+ * optional -- without it the batch runs on the CUDA-core kernel.  With one
+ * LUT set the tensor-core LUT gradient requires its workspace.
  */
 size_t sk_workspace_bytes(int op, int64_t n, int64_t d, int bits, int gpr,
                           int64_t T, int ntask);

@@ -412,3 +412,52 @@ def test_multitask_input_gradient_skewed_and_bad_tasks(monkeypatch):
     ref = oracle.backward_input(c.dy[keep], c.idx, c.lut, c.task[keep])
     bound = oracle.backward_input(np.abs(c.dy[keep]), c.idx, np.abs(c.lut.astype(np.float64)), c.task[keep])
     gc.check_rows(gc.bf16_to_f64(dX)[keep], ref, bound, "dX")
+
+
+# ---------------------------------------------------------------------------
+# several LUT sets on the tensor-core LUT gradient (padded task routing)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("path", ["auto", "simt", "tc"])
+@pytest.mark.parametrize("T,ntask,shape", [(64, 8, (136, 512, 3, 2)), (300, 3, (264, 1376, 2, 1)),
+                                           (1000, 8, (256, 1024, 4, 4)), (513, 2, (512, 2048, 4, 4)),
+                                           (17, 4, (128, 256, 4, 1))])
+def test_multitask_lut_gradient_each_path(monkeypatch, path, T, ntask, shape):
+    sk = _sk()
+    if path != "auto":
+        monkeypatch.setenv("SK_BWD_PATH", path)
+    n, d, bits, gpr = shape
+    c = synth.layer_case(9960 + T, n=n, d=d, bits=bits, gpr=gpr, T=T, ntask=ntask)
+    packed, lut, X, dY, task = gc.dev_case(c)
+    if path == "tc" or (path == "auto" and T >= 64):
+        assert sk.workspace_bytes(sk.SK_OP_BWD_LUT, n, d, bits, gpr, T, ntask) > 0
+    dl = sk.linear_bwd_lut(packed, bits, gpr, X, dY, task, ntask)
+    ref = oracle.backward_lut(c.x, c.dy, c.idx, gpr, 1 << bits, task=c.task, ntask=ntask)
+    gc.check_dlut(dl.cpu().numpy(), ref)
+    assert sk.device_check() == 0
+
+
+def test_multitask_lut_gradient_skewed_empty_bad_and_accumulate():
+    """Most tokens on one set, one set without tokens (its gradient is zero),
+    two tokens with out-of-range ids (left out of every set, flagged), and
+    accumulate = 1 adding onto a previous gradient."""
+    sk = _sk()
+    c = synth.layer_case(9990, n=256, d=1024, bits=4, gpr=4, T=700, ntask=5)
+    c.task[:] = 0
+    c.task[::97] = 2
+    c.task[5] = 4
+    packed, lut, X, dY, task = gc.dev_case(c)
+    task[3] = 9
+    task[400] = -1
+    keep = np.ones(c.T, dtype=bool)
+    keep[[3, 400]] = False
+    ref = oracle.backward_lut(c.x[keep], c.dy[keep], c.idx, 4, 16, task=c.task[keep], ntask=5)
+    assert not ref[1].any() and not ref[3].any()
+    sk.device_check(clear=True)
+    dl = sk.linear_bwd_lut(packed, 4, 4, X, dY, task, 5)
+    assert sk.device_check(clear=True) & sk.SK_CHECK_TASK_RANGE
+    gc.check_dlut(dl.cpu().numpy(), ref)
+    assert not dl[1].any() and not dl[3].any()
+    dl2 = sk.linear_bwd_lut(packed, 4, 4, X, dY, task, 5, out=dl.clone(), accumulate=True)
+    sk.device_check(clear=True)
+    gc.check_dlut(dl2.cpu().numpy(), 2 * ref)
