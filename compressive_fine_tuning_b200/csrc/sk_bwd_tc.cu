@@ -385,6 +385,14 @@ dlut_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant_
     float* bins = reinterpret_cast<float*>(smem + BAR_OFF - K * 128 * 4);  // [K][128], tail of stage memory
     const int tid = threadIdx.x;                                         // 0..127
     const int64_t i = i0 + tid;
+    // the row's index chunks of this column tile, loaded while the MMAs run so
+    // their memory latency is off the binning loop
+    Chunk<BITS> chunks[N / 32];
+#pragma unroll
+    for (int q = 0; q < N / 32; ++q) {
+      const int64_t jc = j0 + 32 * q;
+      if (i < a.n && jc < a.d) chunks[q] = load_chunk<BITS>(a.packed + i * a.row_bytes, jc >> 5);
+    }
     bool have = !*abort_flag && tc::mbar_wait(d_full, 0, a.check) && nsteps > 0;   // no steps: nothing accumulated
     have = __all_sync(0xffffffffu, have);  // tcgen05.ld is warp-collective
     if (have) tc::tc_fence_after();
@@ -404,6 +412,7 @@ dlut_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant_
 #pragma unroll
       for (int c = 0; c < K; ++c) bins[c * 128 + tid] = 0.f;
     };
+#pragma unroll
     for (int q = 0; q < N / 32; ++q) {
       const int64_t jc = j0 + 32 * q;
       if (jc >= a.d) break;
@@ -421,9 +430,8 @@ dlut_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant_
         dirty = false;
       }
       if (i < a.n) {
-        const Chunk<BITS> ch = load_chunk<BITS>(a.packed + i * a.row_bytes, jc >> 5);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) bins[chunk_index<BITS>(ch, e) * 128 + tid] += __uint_as_float(v[e]);
+        for (int e = 0; e < 32; ++e) bins[chunk_index<BITS>(chunks[q], e) * 128 + tid] += __uint_as_float(v[e]);
       }
       dirty = true;
     }
