@@ -154,3 +154,52 @@ LLAMA2_13B = [(5120, 5120)] * 4 + [(13824, 5120)] * 2 + [(5120, 13824)]
 LLAMA3_70B = [(8192, 8192), (1024, 8192), (1024, 8192), (8192, 8192),
               (28672, 8192), (28672, 8192), (8192, 28672)]
 LAYER_NAMES = ["q_proj", "k_proj", "v_proj", "o_proj", "gate_proj", "up_proj", "down_proj"]
+
+
+# ---------------------------------------------------------------------------
+# Sketching-stage inputs ("SpaLLM", section 2.2: dense weights and a small
+# calibration set of layer inputs; the pages use 128 sequences of 2048 tokens)
+# ---------------------------------------------------------------------------
+
+CALIB_COL_SIGMA = 0.5
+
+
+@dataclasses.dataclass
+class SketchCase:
+    """A dense weight and calibration activations for the sketching stage."""
+    n: int
+    d: int
+    s: int
+    theta: np.ndarray       # float32 [n, d], N(0, 0.02)
+    x_bits: np.ndarray      # uint16 (bf16) [s, d]
+
+    @property
+    def x(self) -> np.ndarray:
+        return bf16_bits_to_f64(self.x_bits)
+
+
+def make_calib(rng: np.random.Generator, s: int, d: int) -> np.ndarray:
+    """Raw bf16 bits [s, d]: N(0, 1) activations times a per-column scale
+    exp(N(0, 0.5)), so that columns differ in energy as layer inputs do."""
+    scale = np.exp(rng.normal(0.0, CALIB_COL_SIGMA, size=(1, d)))
+    return f32_to_bf16_bits((rng.normal(0.0, 1.0, size=(s, d)) * scale).astype(np.float32))
+
+
+def sketch_case(seed: int, n: int, d: int, s: int) -> SketchCase:
+    rng = rng_for(seed)
+    theta = rng.normal(0.0, LUT_STD, size=(n, d)).astype(np.float32)
+    return SketchCase(n, d, s, theta, make_calib(rng, s, d))
+
+
+def make_upper(rng: np.random.Generator, d: int) -> np.ndarray:
+    """float64 [d, d] upper-triangular matrix with a positive diagonal
+    (U(0.5, 1.5)) and N(0, 0.3 / sqrt(d)) entries above it: an arbitrary
+    inverse-Hessian factor for testing the mapping step on its own."""
+    u = np.triu(rng.normal(0.0, 0.3 / np.sqrt(d), size=(d, d)), 1)
+    u[np.diag_indices(d)] = rng.uniform(0.5, 1.5, size=d)
+    return u
+
+
+def make_hinv_diag(rng: np.random.Generator, d: int) -> np.ndarray:
+    """float64 [d] positive inverse-Hessian diagonals spread over two decades."""
+    return 10.0 ** rng.uniform(-1.0, 1.0, size=d)

@@ -11,7 +11,10 @@ Sketching" (section 2.2, Eq. 1 and groups per row; section 2.3, multiple LUT
 sets; section 2.4, the identity example) and the "Sketch to Adapt" OpenReview
 discussion (the corrected Eq. 6 and the mapping matrix M).  The LUT update
 (AdamW, SGD, the averaging of shared gradients of section 2.1) is the
-textbook optimizer the pages leave unnamed.  Floating point is
+textbook optimizer the pages leave unnamed.  The sketching stage that
+produces the index map and the first LUTs (section 2.2: calibration Gram
+matrix, weighted Lloyd's algorithm, column-by-column mapping with error
+compensation) is in ``sketching_oracle``.  Floating point is
 float64 throughout; fp16 LUT values and bf16 activations widen exactly.
 
 Parity pins: every function here is pinned by a CPU test against something
@@ -23,4 +26,8 @@ from .sketch_oracle import (  # noqa: F401
     dequant_via_sketch_matrix, forward, backward_input, backward_lut,
     eq6_forward, eq6_backward_lut, bin_counts, trainable_params, lora_params,
     compression_factor, averaged_gradient, adamw_step, sgd_step,
+)
+from .sketching_oracle import (  # noqa: F401
+    gram, damped, inverse_factor, lloyd_init, lloyd_assign, lloyd_update, lloyd,
+    lloyd_luts, sketch_round, sketch_layer, proxy_loss,
 )
