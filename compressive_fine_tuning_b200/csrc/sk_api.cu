@@ -14,6 +14,7 @@
 #include <string>
 
 #include "sk_internal.cuh"
+#include "sk_sketch.cuh"
 
 namespace {
 
@@ -520,6 +521,125 @@ sk_status sk_lut_sgd(float* master, const float* grad, const int32_t* counts, in
   if (st != SK_OK) return st;
   cudaError_t e = sk::launch_sgd(master, grad, counts, total, per_set, lr, lut, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ok() : cuda_fail(e, "SGD kernel launch");
+}
+
+// ---------------------------------------------------------------------------
+// Sketching stage
+// ---------------------------------------------------------------------------
+
+constexpr int64_t kMaxSketchDim = int64_t(1) << 16;
+
+size_t sk_inverse_factor_workspace_bytes(int64_t d) {
+  if (d < 1 || d > kMaxSketchDim) return 0;
+  return sk::inverse_factor_workspace(d);
+}
+
+size_t sk_sketch_round_workspace_bytes(int64_t n, int64_t d) {
+  if (n < 1 || d < 1 || n >= kMaxDim || d > kMaxSketchDim) return 0;
+  return sk::sketch_round_workspace(n, d);
+}
+
+sk_status sk_gram(const uint16_t* X, int64_t s, int64_t d, float* H, int accumulate, sk_stream_t stream) {
+  g_last_error.clear();
+  if (s < 0 || s >= kMaxDim || d < 64 || d > kMaxSketchDim || d % 8)
+    return fail(SK_ERR_INVALID_ARG, "need 0 <= s < 2^31 and 64 <= d <= 65536 with d %% 8 == 0 (s=%lld, d=%lld)",
+                (long long)s, (long long)d);
+  if (!H || (s > 0 && !X)) return fail(SK_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(H) || (X && !aligned16(X))) return fail(SK_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (overlaps(H, (size_t)d * d * 4, X, (size_t)s * d * 2)) return fail(SK_ERR_INVALID_ARG, "output overlaps an input");
+  unsigned int* check = nullptr;
+  sk_status st = device_state(&check);
+  if (st != SK_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
+  if (s == 0) {
+    if (!accumulate) e = cudaMemsetAsync(H, 0, (size_t)d * d * 4, cs);
+  } else {
+    e = sk::launch_gram(X, s, d, H, accumulate, check, cs);
+  }
+  return e == cudaSuccess ? ok() : cuda_fail(e, "Gram kernel launch");
+}
+
+sk_status sk_inverse_factor(const float* H, int64_t d, double damp, double* U, double* hinv_diag, void* workspace,
+                            size_t workspace_bytes, sk_stream_t stream) {
+  g_last_error.clear();
+  if (d < 1 || d > kMaxSketchDim) return fail(SK_ERR_INVALID_ARG, "need 1 <= d <= 65536 (d=%lld)", (long long)d);
+  if (!(damp >= 0.0) || !std::isfinite(damp)) return fail(SK_ERR_INVALID_ARG, "damp must be finite and >= 0");
+  if (!H || !U || !hinv_diag || !workspace) return fail(SK_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(H) || !aligned16(U) || !aligned16(hinv_diag) || !aligned16(workspace))
+    return fail(SK_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  const size_t need = sk::inverse_factor_workspace(d);
+  if (workspace_bytes < need)
+    return fail(SK_ERR_INVALID_ARG, "workspace too small: %zu bytes, need %zu", workspace_bytes, need);
+  const size_t hb = (size_t)d * d * 4, ub = (size_t)d * d * 8, db = (size_t)d * 8;
+  if (overlaps(U, ub, H, hb) || overlaps(hinv_diag, db, H, hb) || overlaps(workspace, need, H, hb) ||
+      overlaps(U, ub, hinv_diag, db) || overlaps(U, ub, workspace, need) || overlaps(hinv_diag, db, workspace, need))
+    return fail(SK_ERR_INVALID_ARG, "buffers overlap");
+  unsigned int* check = nullptr;
+  sk_status st = device_state(&check);
+  if (st != SK_OK) return st;
+  cudaError_t e = sk::launch_inverse_factor(H, d, damp, U, hinv_diag, workspace, check,
+                                            reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ok() : cuda_fail(e, "inverse-factor kernel launch");
+}
+
+static sk_status check_sketch_shape(int bits, int gpr, int64_t n, int64_t d) {
+  if (bits < 2 || bits > 4) return fail(SK_ERR_INVALID_ARG, "bits must be 2, 3 or 4 (got %d)", bits);
+  if (n < 1 || d < 1 || gpr < 1 || n >= kMaxDim || d > kMaxSketchDim || d % gpr)
+    return fail(SK_ERR_INVALID_ARG, "need n, d, gpr >= 1, d <= 65536 and d %% gpr == 0 (n=%lld, d=%lld, gpr=%d)",
+                (long long)n, (long long)d, gpr);
+  return SK_OK;
+}
+
+sk_status sk_lloyd(const float* theta, const double* hinv_diag, int bits, int gpr, int64_t n, int64_t d, int max_iter,
+                   uint16_t* lut, int32_t* iters, sk_stream_t stream) {
+  g_last_error.clear();
+  sk_status st = check_sketch_shape(bits, gpr, n, d);
+  if (st != SK_OK) return st;
+  if (d / gpr > sk::kSketchMaxGroup)
+    return fail(SK_ERR_UNSUPPORTED, "groups of %lld columns; at most %lld", (long long)(d / gpr),
+                (long long)sk::kSketchMaxGroup);
+  if (n * gpr >= kMaxDim) return fail(SK_ERR_INVALID_ARG, "n * gpr must be below 2^31");
+  if (max_iter < 0) return fail(SK_ERR_INVALID_ARG, "max_iter must be >= 0");
+  if (!theta || !hinv_diag || !lut) return fail(SK_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(theta) || !aligned16(hinv_diag) || !aligned16(lut) || (iters && !aligned16(iters)))
+    return fail(SK_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  const size_t lb = (size_t)n * gpr * (1u << bits) * 2, ib = (size_t)n * gpr * 4;
+  const size_t tb = (size_t)n * d * 4, hb = (size_t)d * 8;
+  if (overlaps(lut, lb, theta, tb) || overlaps(lut, lb, hinv_diag, hb) ||
+      (iters && (overlaps(iters, ib, theta, tb) || overlaps(iters, ib, hinv_diag, hb) || overlaps(iters, ib, lut, lb))))
+    return fail(SK_ERR_INVALID_ARG, "buffers overlap");
+  unsigned int* check = nullptr;
+  st = device_state(&check);
+  if (st != SK_OK) return st;
+  cudaError_t e = sk::launch_lloyd(theta, hinv_diag, bits, gpr, n, d, max_iter, lut, iters,
+                                   reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ok() : cuda_fail(e, "Lloyd kernel launch");
+}
+
+sk_status sk_sketch_round(const float* theta, const double* U, const uint16_t* lut, int bits, int gpr, int64_t n,
+                          int64_t d, uint8_t* idx, void* workspace, size_t workspace_bytes, sk_stream_t stream) {
+  g_last_error.clear();
+  sk_status st = check_sketch_shape(bits, gpr, n, d);
+  if (st != SK_OK) return st;
+  if (n > (int64_t)65535 * 64) return fail(SK_ERR_UNSUPPORTED, "at most 4194240 rows");
+  if (!theta || !U || !lut || !idx || !workspace) return fail(SK_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(theta) || !aligned16(U) || !aligned16(lut) || !aligned16(idx) || !aligned16(workspace))
+    return fail(SK_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  const size_t need = sk::sketch_round_workspace(n, d);
+  if (workspace_bytes < need)
+    return fail(SK_ERR_INVALID_ARG, "workspace too small: %zu bytes, need %zu", workspace_bytes, need);
+  const size_t xb = (size_t)n * d, tb = xb * 4, ub = (size_t)d * d * 8, lb = (size_t)n * gpr * (1u << bits) * 2;
+  if (overlaps(idx, xb, theta, tb) || overlaps(idx, xb, U, ub) || overlaps(idx, xb, lut, lb) ||
+      overlaps(idx, xb, workspace, need) || overlaps(workspace, need, theta, tb) || overlaps(workspace, need, U, ub) ||
+      overlaps(workspace, need, lut, lb))
+    return fail(SK_ERR_INVALID_ARG, "buffers overlap");
+  unsigned int* check = nullptr;
+  st = device_state(&check);
+  if (st != SK_OK) return st;
+  cudaError_t e = sk::launch_sketch_round(theta, U, lut, bits, gpr, n, d, idx, workspace, check,
+                                          reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ok() : cuda_fail(e, "mapping kernel launch");
 }
 
 sk_status sk_device_check(uint32_t* flags, int clear, sk_stream_t stream) {

@@ -19,12 +19,16 @@ SK_OK = 0
 SK_OP_FWD, SK_OP_BWD_INPUT, SK_OP_BWD_LUT = 0, 1, 2
 SK_CHECK_TASK_RANGE = 1
 SK_CHECK_INDEX_RANGE = 2
+SK_CHECK_TIMEOUT = 4
+SK_CHECK_NOT_SPD = 8
+SK_CHECK_LUT_ORDER = 16
 
 EXPORTED = (
     "sk_abi_version", "sk_status_string", "sk_last_error", "sk_packed_row_bytes", "sk_packed_bytes",
     "sk_pack", "sk_unpack", "sk_dequant", "sk_workspace_bytes", "sk_linear_fwd", "sk_linear_bwd_input",
     "sk_linear_bwd_lut", "sk_linear_bwd_lut_noalloc", "sk_bin_counts", "sk_lut_adamw", "sk_lut_sgd",
-    "sk_device_check",
+    "sk_device_check", "sk_inverse_factor_workspace_bytes", "sk_sketch_round_workspace_bytes", "sk_gram",
+    "sk_inverse_factor", "sk_lloyd", "sk_sketch_round",
 )
 
 
@@ -39,6 +43,7 @@ def _load() -> ctypes.CDLL:
         raise ImportError(f"{_LIB_PATH} is missing: build it with `python -m compressive_fine_tuning_b200.build`")
     lib = ctypes.CDLL(_LIB_PATH)
     vp, i64, i32, sz, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+    f64 = ctypes.c_double
     sigs = {
         "sk_abi_version": ([], i32),
         "sk_status_string": ([i32], ctypes.c_char_p),
@@ -57,6 +62,12 @@ def _load() -> ctypes.CDLL:
         "sk_lut_adamw": ([vp, vp, vp, vp, vp, i32, i64, i32, i32, f32, f32, f32, f32, f32, i32, vp, vp], i32),
         "sk_lut_sgd": ([vp, vp, vp, i32, i64, i32, i32, f32, vp, vp], i32),
         "sk_device_check": ([ctypes.POINTER(ctypes.c_uint32), i32, vp], i32),
+        "sk_inverse_factor_workspace_bytes": ([i64], sz),
+        "sk_sketch_round_workspace_bytes": ([i64, i64], sz),
+        "sk_gram": ([vp, i64, i64, vp, i32, vp], i32),
+        "sk_inverse_factor": ([vp, i64, f64, vp, vp, vp, sz, vp], i32),
+        "sk_lloyd": ([vp, vp, i32, i32, i64, i64, i32, vp, vp, vp], i32),
+        "sk_sketch_round": ([vp, vp, vp, i32, i32, i64, i64, vp, vp, sz, vp], i32),
     }
     for name, (args, res) in sigs.items():
         fn = getattr(lib, name)
@@ -266,6 +277,77 @@ def lut_sgd_(master: torch.Tensor, grad: torch.Tensor, bits: int, lr: float, cou
         raise ValueError("lut must be contiguous fp16 of the master's shape")
     _check(lib.sk_lut_sgd(_ptr(master), _ptr(grad), _ptr(counts), ntask, n, gpr, bits, lr, _ptr(lut),
                           _stream(master.device)))
+
+
+# ---------------------------------------------------------------------------
+# Sketching stage: dense weight + calibration activations -> index map + LUTs
+# ---------------------------------------------------------------------------
+
+def gram(X: torch.Tensor, H: Optional[torch.Tensor] = None, accumulate: bool = False) -> torch.Tensor:
+    """H = X^T X (fp32 [d, d]) of bf16 calibration activations X [s, d];
+    H += X^T X when accumulate."""
+    _need(X, torch.bfloat16, "X", 2)
+    s, d = X.shape
+    if H is None:
+        H = torch.empty((d, d), dtype=torch.float32, device=X.device)
+    _need(H, torch.float32, "H", 2)
+    _check(lib.sk_gram(_ptr(X), s, d, _ptr(H), int(accumulate), _stream(X.device)))
+    return H
+
+
+def inverse_factor(H: torch.Tensor, damp: float = 0.01):
+    """(U, hinv_diag): the upper factor U of the damped H^-1 (H^-1 = U^T U,
+    float64 [d, d]) and the diagonal of H^-1 (float64 [d])."""
+    _need(H, torch.float32, "H", 2)
+    d = H.shape[0]
+    U = torch.empty((d, d), dtype=torch.float64, device=H.device)
+    hd = torch.empty(d, dtype=torch.float64, device=H.device)
+    nb = int(lib.sk_inverse_factor_workspace_bytes(d))
+    ws = torch.empty(max(nb, 1), dtype=torch.uint8, device=H.device)
+    _check(lib.sk_inverse_factor(_ptr(H), d, float(damp), _ptr(U), _ptr(hd), _ptr(ws), nb, _stream(H.device)))
+    return U, hd
+
+
+def lloyd(theta: torch.Tensor, hinv_diag: torch.Tensor, bits: int, gpr: int, max_iter: int = 100):
+    """(lut fp16 [n, gpr, 2^bits], updates run int32 [n, gpr]): weighted
+    Lloyd's centroids of every (row, group) of theta (fp32 [n, d])."""
+    _need(theta, torch.float32, "theta", 2)
+    _need(hinv_diag, torch.float64, "hinv_diag", 1)
+    n, d = theta.shape
+    lut = torch.empty((n, gpr, 1 << bits), dtype=torch.float16, device=theta.device)
+    iters = torch.empty((n, gpr), dtype=torch.int32, device=theta.device)
+    _check(lib.sk_lloyd(_ptr(theta), _ptr(hinv_diag), bits, gpr, n, d, max_iter, _ptr(lut), _ptr(iters),
+                        _stream(theta.device)))
+    return lut, iters
+
+
+def sketch_round(theta: torch.Tensor, U: torch.Tensor, lut: torch.Tensor, bits: int) -> torch.Tensor:
+    """Index map (uint8 [n, d]) of theta against the ascending fp16 LUTs
+    [n, gpr, 2^bits], with error compensation through U."""
+    _need(theta, torch.float32, "theta", 2)
+    _need(U, torch.float64, "U", 2)
+    _need(lut, torch.float16, "lut", 3)
+    n, d = theta.shape
+    gpr = lut.shape[1]
+    idx = torch.empty((n, d), dtype=torch.uint8, device=theta.device)
+    nb = int(lib.sk_sketch_round_workspace_bytes(n, d))
+    ws = torch.empty(max(nb, 1), dtype=torch.uint8, device=theta.device)
+    _check(lib.sk_sketch_round(_ptr(theta), _ptr(U), _ptr(lut), bits, gpr, n, d, _ptr(idx), _ptr(ws), nb,
+                               _stream(theta.device)))
+    return idx
+
+
+def sketch_layer(theta: torch.Tensor, X: torch.Tensor, bits: int, gpr: int, damp: float = 0.01,
+                 max_iter: int = 100, H: Optional[torch.Tensor] = None):
+    """The sketching stage of one layer: (packed index map, fp16 LUTs
+    [n, gpr, 2^bits], index map uint8 [n, d]).  H, when given, is the
+    calibration Gram matrix already accumulated (X is then ignored)."""
+    if H is None:
+        H = gram(X)
+    U, hd = inverse_factor(H, damp)
+    lut, _ = lloyd(theta, hd, bits, gpr, max_iter)
+    idx = sketch_round(theta, U, lut, bits)
+    return pack(idx, bits), lut, idx
 
 
 class SketchedLinearFunction(torch.autograd.Function):

@@ -79,6 +79,10 @@ typedef enum {
 #define SK_CHECK_INDEX_RANGE 2u  /* sk_pack saw an index >= 2^bits             */
 #define SK_CHECK_TIMEOUT 4u      /* a kernel gave up waiting on its own pipeline
                                     (an internal error; its outputs are invalid) */
+#define SK_CHECK_NOT_SPD 8u      /* sk_inverse_factor met a pivot <= 0: the damped
+                                    Gram matrix is not positive definite       */
+#define SK_CHECK_LUT_ORDER 16u   /* sk_sketch_round was given a LUT that is not
+                                    ascending                                   */
 
 /* Operation selectors for sk_workspace_bytes. */
 #define SK_OP_FWD 0
@@ -242,6 +246,60 @@ sk_status sk_lut_adamw(float* master, float* m, float* v, const float* grad, con
                        float weight_decay, int step, uint16_t* lut, sk_stream_t stream);
 sk_status sk_lut_sgd(float* master, const float* grad, const int32_t* counts, int ntask, int64_t n, int gpr,
                      int bits, float lr, uint16_t* lut, sk_stream_t stream);
+
+/*
+ * Sketching stage ("SpaLLM: Unified Compressive Adaptation of LLMs with
+ * Sketching", section 2.2; "Sketch to Adapt" OpenReview discussion, concern
+ * 1): from a dense weight Theta (float32 [n][d]) and calibration activations
+ * X (bf16 [s][d]; the pages use 128 sequences of 2048 tokens) to the index
+ * map and the first fp16 LUTs.  Run once per layer; every buffer is device
+ * memory owned by the caller; nothing is allocated.  The usual chain is
+ *   sk_gram -> sk_inverse_factor -> sk_lloyd -> sk_sketch_round -> sk_pack.
+ *
+ * sk_gram: H (float32 [d][d]) = X^T X, or H += X^T X when accumulate != 0
+ * (calibration data may come in batches).  Tensor cores, fp32 accumulation.
+ * 0 <= s < 2^31, 64 <= d <= 65536, d % 8 == 0.  s == 0 zeroes H (or leaves
+ * it when accumulating).
+ *
+ * sk_inverse_factor: damping, then the inverse factor in float64.  A zero
+ * diagonal entry of H counts as 1, then damp * mean(diag H) is added to the
+ * diagonal (the pages are silent on damping; this follows the error-
+ * compensated rounding they cite).  Only the upper triangle of H is read.
+ * Outputs U (float64 [d][d], upper triangular, H^-1 = U^T U) and hinv_diag
+ * (float64 [d], the diagonal of H^-1).  workspace: at least
+ * sk_inverse_factor_workspace_bytes(d) bytes.  A damped H that is not
+ * positive definite sets SK_CHECK_NOT_SPD (the outputs then hold NaNs).
+ *
+ * sk_lloyd: weighted Lloyd's algorithm per (row, group), weights
+ * 1 / hinv_diag[j], k = 2^bits centroids started evenly over the group's
+ * [min, max]; a value joins the centroid whose float32 midpoints bracket it
+ * (a value on a midpoint goes to the lower one), a centroid becomes the
+ * float64 weighted mean of its members rounded to float32 (an empty cluster
+ * keeps its centroid); stops when an update moves no value, or after
+ * max_iter updates.  Writes lut (fp16 bits [n][gpr][k], ascending) and, if
+ * iters is not NULL, the updates run per (row, group) (int32 [n][gpr]).
+ * d % gpr == 0 and d / gpr <= 16384 (else SK_ERR_UNSUPPORTED).  theta must
+ * be finite.
+ *
+ * sk_sketch_round: the index map (uint8 [n][d], values < 2^bits).  Columns
+ * are mapped in order: column j of every row goes to the nearest entry of
+ * its group's LUT (float32 midpoints, ties to the lower entry) of its current
+ * value w_j, and the later columns c of the row move by
+ * -(w_j - q_j) / U_jj * U_jc (the Optimal Brain Surgeon update over the
+ * columns not yet mapped; the reading of the discussion's Eq. 13).  Values
+ * are carried in float64.  lut: fp16 bits [n][gpr][k], ascending per group
+ * (a descending pair sets SK_CHECK_LUT_ORDER).  workspace: at least
+ * sk_sketch_round_workspace_bytes(n, d) bytes.
+ */
+size_t sk_inverse_factor_workspace_bytes(int64_t d);
+size_t sk_sketch_round_workspace_bytes(int64_t n, int64_t d);
+sk_status sk_gram(const uint16_t* X, int64_t s, int64_t d, float* H, int accumulate, sk_stream_t stream);
+sk_status sk_inverse_factor(const float* H, int64_t d, double damp, double* U, double* hinv_diag, void* workspace,
+                            size_t workspace_bytes, sk_stream_t stream);
+sk_status sk_lloyd(const float* theta, const double* hinv_diag, int bits, int gpr, int64_t n, int64_t d, int max_iter,
+                   uint16_t* lut, int32_t* iters, sk_stream_t stream);
+sk_status sk_sketch_round(const float* theta, const double* U, const uint16_t* lut, int bits, int gpr, int64_t n,
+                          int64_t d, uint8_t* idx, void* workspace, size_t workspace_bytes, sk_stream_t stream);
 
 /*
  * sk_device_check: synchronises `stream`, stores the device check word

@@ -165,3 +165,60 @@ def test_lut_update_without_device_fails_loudly():
         pytest.skip("a CUDA device is present")
     assert _adamw() in (SK_ERR_CUDA, SK_ERR_UNSUPPORTED)
     assert sk.lib.sk_lut_sgd(A, B, None, 1, 8, 2, 4, 0.1, None, None) in (SK_ERR_CUDA, SK_ERR_UNSUPPORTED)
+
+
+E = ctypes.c_void_p(0x50000000)
+F = ctypes.c_void_p(0x60000000)
+
+
+def test_sketch_workspace_sizes():
+    L = sk.lib
+    assert L.sk_inverse_factor_workspace_bytes(4096) >= 4096 * 4096 * 8
+    assert L.sk_inverse_factor_workspace_bytes(0) == 0
+    assert L.sk_inverse_factor_workspace_bytes(1 << 17) == 0
+    assert L.sk_sketch_round_workspace_bytes(4096, 4096) >= 4096 * 4096 * 8
+    assert L.sk_sketch_round_workspace_bytes(0, 64) == 0
+
+
+def test_sketch_validation():
+    L = sk.lib
+    big = 1 << 30
+    # Gram: d >= 64 and a multiple of 8, pointers, aligned, no overlap
+    assert L.sk_gram(A, 16, 60, B, 0, None) == SK_ERR_INVALID_ARG
+    assert L.sk_gram(A, 16, 100, B, 0, None) == SK_ERR_INVALID_ARG
+    assert L.sk_gram(A, -1, 64, B, 0, None) == SK_ERR_INVALID_ARG
+    assert L.sk_gram(None, 16, 64, B, 0, None) == SK_ERR_INVALID_ARG
+    assert L.sk_gram(A, 16, 64, ctypes.c_void_p(0x20000008), 0, None) == SK_ERR_INVALID_ARG
+    assert L.sk_gram(A, 16, 64, ctypes.c_void_p(0x10000000 + 64), 0, None) == SK_ERR_INVALID_ARG
+    # inverse factor: damp, workspace size, overlaps
+    ws = L.sk_inverse_factor_workspace_bytes(64)
+    assert L.sk_inverse_factor(A, 64, -0.1, B, C, D, ws, None) == SK_ERR_INVALID_ARG
+    assert L.sk_inverse_factor(A, 64, float("inf"), B, C, D, ws, None) == SK_ERR_INVALID_ARG
+    assert L.sk_inverse_factor(A, 64, 0.01, B, C, D, ws - 1, None) == SK_ERR_INVALID_ARG
+    assert L.sk_inverse_factor(A, 64, 0.01, B, ctypes.c_void_p(0x20000000 + 64), D, ws, None) == SK_ERR_INVALID_ARG
+    assert L.sk_inverse_factor(A, 0, 0.01, B, C, D, big, None) == SK_ERR_INVALID_ARG
+    # Lloyd: bits, gpr dividing d, group length, max_iter
+    assert L.sk_lloyd(A, B, 5, 1, 8, 64, 10, C, None, None) == SK_ERR_INVALID_ARG
+    assert L.sk_lloyd(A, B, 4, 3, 8, 64, 10, C, None, None) == SK_ERR_INVALID_ARG
+    assert L.sk_lloyd(A, B, 4, 1, 8, 32768, 10, C, None, None) == SK_ERR_UNSUPPORTED
+    assert L.sk_lloyd(A, B, 4, 1, 8, 64, -1, C, None, None) == SK_ERR_INVALID_ARG
+    assert L.sk_lloyd(A, B, 4, 1, 8, 64, 10, ctypes.c_void_p(0x10000000 + 16), None, None) == SK_ERR_INVALID_ARG
+    # mapping: workspace size, overlaps
+    wr = L.sk_sketch_round_workspace_bytes(8, 64)
+    assert L.sk_sketch_round(A, B, C, 4, 1, 8, 64, D, E, wr - 1, None) == SK_ERR_INVALID_ARG
+    assert L.sk_sketch_round(A, B, C, 4, 1, 8, 64, None, E, wr, None) == SK_ERR_INVALID_ARG
+    assert L.sk_sketch_round(A, B, C, 4, 1, 8, 64, ctypes.c_void_p(0x30000000 + 16), E, wr, None) == SK_ERR_INVALID_ARG
+    assert L.sk_sketch_round(A, B, C, 4, 2, 8, 63, D, E, wr, None) == SK_ERR_INVALID_ARG
+
+
+def test_sketch_without_device_fails_loudly():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present")
+    L = sk.lib
+    assert L.sk_gram(A, 16, 64, B, 0, None) in (SK_ERR_CUDA, SK_ERR_UNSUPPORTED)
+    assert L.sk_inverse_factor(A, 64, 0.01, B, C, D, L.sk_inverse_factor_workspace_bytes(64), None) in (
+        SK_ERR_CUDA, SK_ERR_UNSUPPORTED)
+    assert L.sk_lloyd(A, B, 4, 1, 8, 64, 10, C, None, None) in (SK_ERR_CUDA, SK_ERR_UNSUPPORTED)
+    assert L.sk_sketch_round(A, B, C, 4, 1, 8, 64, D, E, L.sk_sketch_round_workspace_bytes(8, 64), None) in (
+        SK_ERR_CUDA, SK_ERR_UNSUPPORTED)
