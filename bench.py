@@ -62,6 +62,18 @@ WORKLOADS = {
                              desc="LLaMA-3-70B-shaped multi-task prefill, 7 layers, 4-bit, GPR=4, 8 LUT sets, T=4096"),
 }
 
+# The sketching stage (SpaLLM section 2.2) of one LLaMA-2-7B block: four
+# distinct layer inputs (q/k/v share one, gate/up share one), seven weights,
+# the pages' calibration set of 128 sequences of 2048 tokens.
+SKETCH_METRIC = "sketching stage: weights sketched per second (Gram, inverse factor, weighted Lloyd, mapping)"
+SKETCH_INPUTS = (("qkv", (0, 1, 2)), ("o", (3,)), ("gate_up", (4, 5)), ("down", (6,)))
+WORKLOADS["sketch7b"] = dict(shapes="LLAMA2_7B", bits=4, gpr=8, batches=(128 * 2048,), ntask=1, ops=("sketch",),
+                             desc="sketching stage of one LLaMA-2-7B block: 128x2048 calibration tokens, "
+                                  "4-bit, GPR=8, damp 0.01, at most 100 Lloyd updates")
+# float64 FMA lanes per SM per cycle on B200 (NVIDIA's 37 TFLOP/s FP64 at the
+# 1965 MHz boost clock over 148 SMs); the fp64 stages report against this
+FP64_LANES_PER_SM = 64
+
 L2_BYTES = 126 * 1024 * 1024
 # Integer-ALU cost of one 4-bit lookup (byte-permute network) and the integer
 # pipe's issue rate per SM on B200, measured with a throughput probe.
@@ -510,6 +522,226 @@ def run_ours(args, w, rank, world, device):
     return res
 
 
+# ---------------------------------------------------------------------------
+# the sketching stage (dense weights + calibration activations -> sketch)
+# ---------------------------------------------------------------------------
+
+def sketch_cpu_baseline(budget_rows=32, tokens=4096, seed=0):
+    """The oracle's sketching stage on a bounded sample: the q_proj input with
+    `tokens` calibration tokens (Gram matrix and inverse factor of the full
+    4096-wide input), then Lloyd and the mapping for `budget_rows` rows."""
+    import oracle
+    from compressive_fine_tuning_b200 import synth
+    n, d = synth.LLAMA2_7B[0]
+    c = synth.sketch_case(seed + 777, budget_rows, d, tokens)
+    t0 = time.perf_counter()
+    h = oracle.damped(oracle.gram(c.x), 0.01)
+    u, hd = oracle.inverse_factor(h)
+    lut = oracle.lloyd_luts(c.theta, hd, 4, 8, 100)
+    oracle.sketch_round(c.theta, u, lut)
+    el = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    sample = (f"q_proj input (d={d}): Gram of {tokens} tokens, inverse factor, then Lloyd and mapping "
+              f"of {budget_rows} of the {n} rows")
+    return budget_rows * d, el, cores, sample
+
+
+def sketch_inputs():
+    """The distinct layer inputs and the weights that read them (restricted to
+    --layers when given)."""
+    out = []
+    for name, members in SKETCH_INPUTS:
+        m = tuple(li for li in members if _LAYER_SUBSET is None or li in _LAYER_SUBSET)
+        if m:
+            out.append((name, m))
+    return out
+
+
+def run_sketch(args, w, rank, device):
+    """Time the sketching stage of one 7B block per step; stage boundaries
+    carry CUDA events on the launching stream."""
+    import torch
+    from compressive_fine_tuning_b200 import sk, synth
+    shapes = synth.LLAMA2_7B
+    bits, gpr, s_tok = w["bits"], w["gpr"], w["batches"][0]
+    g = torch.Generator(device=device).manual_seed(args.seed * 1000 + rank)
+    # calibration activations: N(0, 1) times a per-column scale exp(N(0, 0.5)), bf16
+    X = {}
+    for name, members in sketch_inputs():
+        d = shapes[members[0]][1]
+        scale = torch.exp(torch.randn(d, generator=g, device=device) * synth.CALIB_COL_SIGMA)
+        X[name] = (torch.randn((s_tok, d), generator=g, device=device) * scale).to(torch.bfloat16)
+    theta = {li: torch.randn((shapes[li][0], shapes[li][1]), generator=g, device=device) * synth.LUT_STD
+             for _, members in sketch_inputs() for li in members}
+    stage_names = ("gram", "factor", "lloyd", "round")
+
+    def step(evs=None, host=None):
+        out = []
+        mark = (lambda nm: evs.append((nm, torch.cuda.Event(enable_timing=True)))) if evs is not None else None
+        for name, members in sketch_inputs():
+            if mark: mark("gram"); evs[-1][1].record()
+            xin = X[name] if host is None else host["X"][name].to(device, non_blocking=True)
+            H = sk.gram(xin)
+            if mark: mark("factor"); evs[-1][1].record()
+            U, hd = sk.inverse_factor(H, 0.01)
+            for li in members:
+                th = theta[li] if host is None else host["theta"][li].to(device, non_blocking=True)
+                if mark: mark("lloyd"); evs[-1][1].record()
+                lut, _ = sk.lloyd(th, hd, bits, gpr, 100)
+                if mark: mark("round"); evs[-1][1].record()
+                idx = sk.sketch_round(th, U, lut, bits)
+                out.append((sk.pack(idx, bits), lut))
+        if mark: mark("end"); evs[-1][1].record()
+        return out
+
+    K, W = args.steps, args.warmup
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize(device)
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    all_evs = []
+    t0 = torch.cuda.Event(enable_timing=True); t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    t0.record()
+    for _ in range(K):
+        evs = []
+        step(evs)
+        all_evs.append(evs)
+    t1.record()
+    torch.cuda.synchronize(device)
+    clocks = sampler.stop() if sampler else None
+    ms = t0.elapsed_time(t1)
+    per_stage = {nm: 0.0 for nm in stage_names}
+    for evs in all_evs:
+        for (nm, e), (_, e2) in zip(evs[:-1], evs[1:]):
+            per_stage[nm] += e.elapsed_time(e2)
+    used = [li for _, m in sketch_inputs() for li in m]
+    weights = sum(shapes[li][0] * shapes[li][1] for li in used)
+    # algorithmic work per stage and step
+    work = {"gram": sum(2.0 * s_tok * shapes[m[0]][1] ** 2 for _, m in sketch_inputs()),
+            "factor": sum(2.0 / 3.0 * shapes[m[0]][1] ** 3 for _, m in sketch_inputs()),
+            "round": sum(float(shapes[li][0]) * shapes[li][1] ** 2 for li in used)}
+    res = dict(ms=ms, per_stage=per_stage, work=work, weights=weights, clocks=clocks)
+    if not args.no_e2e:
+        host = {"X": {k: v.cpu().pin_memory() for k, v in X.items()},
+                "theta": {li: t.cpu().pin_memory() for li, t in theta.items()}}
+        step(host=host)
+        torch.cuda.synchronize(device)
+        h2d = sum(v.numel() * v.element_size() for v in host["X"].values()) + \
+            sum(t.numel() * t.element_size() for t in host["theta"].values())
+        e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        out = step(host=host)
+        back = [(p.cpu(), l.cpu()) for p, l in out]
+        e1.record()
+        torch.cuda.synchronize(device)
+        d2h = sum(p.numel() * p.element_size() + l.numel() * l.element_size() for p, l in back)
+        res["e2e"] = dict(ms=e0.elapsed_time(e1), h2d=h2d, d2h=d2h)
+    return res
+
+
+def main_sketch(args, w, world, rank, local):
+    pk = peaks()
+    config = {"workload": args.workload, "desc": w["desc"], "bits": w["bits"], "gpr": w["gpr"],
+              "calibration_tokens": w["batches"][0], "layers": [list(x) for x in layer_shapes(w)],
+              "inputs": {nm: list(m) for nm, m in sketch_inputs()},
+              "parallelism": "single" if world == 1 else f"replicas{world} (one block per rank)",
+              "l2": "calibration activations (2-6 GB per input) and weights exceed L2"}
+    unit = "weights/s"
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        best = None
+        for _ in range(max(1, min(args.steps, 2))):
+            wts, el, cores, sample = sketch_cpu_baseline(seed=args.seed)
+            best = el if best is None else min(best, el)
+        v = wts / best
+        print(json.dumps({"impl": "reference", "metric": SKETCH_METRIC, "value": v, "unit": unit, "n_gpus": 1,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": best * 1e3,
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                          "data": "synthetic", "config": config,
+                          "cpu_baseline": {"value": v, "unit": unit, "cores": cores, "kind": "oracle", "sample": sample},
+                          "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+        return 0
+    import torch
+    import torch.distributed as dist
+    import datetime
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    device = torch.device("cuda", torch.cuda.current_device())
+    if world > 1:
+        dist.barrier()
+    res = run_sketch(args, w, rank, device)
+    ms = res["ms"]
+    if world > 1:
+        t = torch.tensor([ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    K = args.steps
+    step_ms = ms / K
+    st = {k: v / K for k, v in res["per_stage"].items()}
+    dom = max(st, key=st.get)
+    mhz = (res["clocks"] or {}).get("sm_mhz") or 1965.0
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    fp64_peak = sms * FP64_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
+    rates = {}
+    for k, v in st.items():
+        if k in res["work"]:
+            rates[k] = res["work"][k] / (v / 1e3) / 1e12
+    if dom == "gram":
+        roof = {"bound": "tensor", "achieved": rates["gram"], "peak": pk["bf16_sus"], "unit": "TFLOP/s",
+                "frac": rates["gram"] / pk["bf16_sus"], "kernel": "gram_tc_kernel",
+                "peak_source": pk["source"] + " bf16_tflops_sustained"}
+    elif dom in ("factor", "round"):
+        roof = {"bound": "alu", "achieved": rates[dom], "peak": fp64_peak, "unit": "TFLOP/s (fp64)",
+                "frac": rates[dom] / fp64_peak,
+                "kernel": "gemm_sub_f64_kernel (" + ("Cholesky and triangular inverse" if dom == "factor"
+                                                     else "mapping: later-column compensation") + ")",
+                "peak_source": f"{FP64_LANES_PER_SM} fp64 FMA lanes/cycle/SM (nominal) x SMs x median SM clock"}
+    else:
+        roof = {"bound": "alu", "achieved": None, "peak": None, "unit": None, "frac": None, "kernel": "lloyd_kernel"}
+    roof["traffic"] = None
+    roof["share"] = st[dom] / step_ms
+    roof["stages_ms"] = st
+    roof["stage_rates_tflops"] = rates
+    roof["fp64_peak_tflops"] = fp64_peak
+    n_launch = 0
+    from compressive_fine_tuning_b200 import synth
+    shapes = synth.LLAMA2_7B
+    for _, members in sketch_inputs():
+        d = shapes[members[0]][1]
+        nb = (d + 63) // 64
+        n_launch += 1 + 2 + 3 * nb - 2 + 1 + 2 * nb - 1 + 2   # Gram; damping; Cholesky; identity; inverse; reverse, norms
+        for li in members:
+            nbl = (shapes[li][1] + 63) // 64
+            n_launch += 1 + 1 + 2 * nbl - 1 + 1                 # Lloyd; copy; mapping blocks and GEMMs; pack
+    line = {"metric": SKETCH_METRIC, "value": res["weights"] * world / (step_ms / 1e3), "unit": unit,
+            "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+            "roofline": roof, "gpu_launches": n_launch * K, "clocks": res["clocks"]}
+    if "e2e" in res:
+        e = res["e2e"]
+        line["e2e"] = {"value": res["weights"] / (e["ms"] / 1e3), "unit": unit, "h2d_bytes_per_step": e["h2d"],
+                       "d2h_bytes_per_step": e["d2h"]}
+    if not args.no_cpu_baseline:
+        wts, el, cores, sample = sketch_cpu_baseline(seed=args.seed)
+        line["cpu_baseline"] = {"value": wts / el, "unit": unit, "cores": cores, "kind": "oracle", "sample": sample}
+    print(json.dumps(line))
+    return 0
+
+
 def fmt_units(w):
     hbm = is_hbm_bound(w)
     return ("GB/s", 1e9) if hbm else ("TFLOP/s", 1e12)
@@ -524,6 +756,8 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if w["ops"] == ("sketch",):
+        return main_sketch(args, w, world, rank, local)
     unit, scale = fmt_units(w)
     pk = peaks()
     config = {"workload": args.workload, "desc": w["desc"], "bits": w["bits"], "gpr": w["gpr"],

@@ -233,11 +233,8 @@ __global__ void __launch_bounds__(256) potrf_diag_kernel(double* __restrict__ A,
     const double piv = a[c][c];
     for (int r = c + 1 + (int)threadIdx.x; r < kb; r += blockDim.x) a[r][c] /= piv;
     __syncthreads();
-    const int m = kb - c - 1;
-    for (int e = threadIdx.x; e < m * m; e += blockDim.x) {
-      const int r = c + 1 + e / m, q = c + 1 + e % m;
-      if (q <= r) a[r][q] -= a[r][c] * a[q][c];
-    }
+    for (int r = c + 1 + (int)(threadIdx.x >> 4); r < kb; r += 16)
+      for (int q = c + 1 + (int)(threadIdx.x & 15); q <= r; q += 16) a[r][q] -= a[r][c] * a[q][c];
     __syncthreads();
   }
   for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
@@ -248,7 +245,7 @@ __global__ void __launch_bounds__(256) potrf_diag_kernel(double* __restrict__ A,
 
 // Panel below a factored diagonal block: row r of A[k0+NB:, k0:k0+NB] becomes
 // x with x L_kk^T = a (forward substitution), one thread per row
-__global__ void __launch_bounds__(128) trsm_panel_kernel(double* __restrict__ A, int64_t d, int64_t k0) {
+__global__ void __launch_bounds__(64) trsm_panel_kernel(double* __restrict__ A, int64_t d, int64_t k0) {
   __shared__ double l[NB][NB + 1];
   for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
     const int r = e / NB, c = e % NB;
@@ -261,73 +258,111 @@ __global__ void __launch_bounds__(128) trsm_panel_kernel(double* __restrict__ A,
   double x[NB];
 #pragma unroll
   for (int c = 0; c < NB; ++c) x[c] = row[c];
+  // the dot products run as four interleaved partial sums (shorter dependency chains)
 #pragma unroll
   for (int c = 0; c < NB; ++c) {
-    double v = x[c];
+    double p[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
-    for (int q = 0; q < c; ++q) v -= x[q] * l[c][q];
-    x[c] = v / l[c][c];
+    for (int q = 0; q < c; ++q) p[q & 3] = fma(x[q], l[c][q], p[q & 3]);
+    x[c] = (x[c] - ((p[0] + p[1]) + (p[2] + p[3]))) / l[c][c];
   }
 #pragma unroll
   for (int c = 0; c < NB; ++c) row[c] = x[c];
 }
 
-// C[m][n] -= A[m][NB] * B, with B(k, c) = B[c][k] (BT) or B[k][c]; 64 x 64
-// output tiles, 4 x 4 per thread; LOWER skips the tiles above the diagonal
+// C[m][n] -= A[m][NB] * B, with B(k, c) = B[c][k] (BT) or B[k][c].  128 x 128
+// output tiles, 8 x 8 per thread (rows ty*4 + {0..3} and 64 + ty*4 + {0..3},
+// likewise the columns), K in chunks of 16 staged k-major in shared memory:
+// per k a thread loads 8 + 8 doubles for 64 FMAs, which keeps the float64
+// FMA pipe, not shared memory, the limit.  LOWER skips the tiles above the
+// diagonal.
+constexpr int GT = 128, GK = 16, GP = GT + 2;   // tile, K chunk, padded row of a staged chunk
+
 template <bool BT, bool LOWER>
-__global__ void __launch_bounds__(256) gemm_sub_f64_kernel(const double* __restrict__ Ap, int64_t lda,
-                                                           const double* __restrict__ Bp, int64_t ldb,
-                                                           double* __restrict__ C, int64_t ldc, int64_t m, int64_t n) {
-  constexpr int TM = 64, TN = 64, KH = 32;
+__global__ void __launch_bounds__(256, 1) gemm_sub_f64_kernel(const double* __restrict__ Ap, int64_t lda,
+                                                              const double* __restrict__ Bp, int64_t ldb,
+                                                              double* __restrict__ C, int64_t ldc, int64_t m,
+                                                              int64_t n, int vec_a, int vec_b) {
   if (LOWER && blockIdx.x > blockIdx.y) return;
-  __shared__ double As[KH][TM + 1];   // [k][row]
-  __shared__ double Bs[KH][TN + 1];   // [k][col]
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  const int64_t r0 = (int64_t)blockIdx.y * TM, c0 = (int64_t)blockIdx.x * TN;
-  double acc[4][4];
+  __shared__ __align__(16) double As[GK][GP];   // [k][row]
+  __shared__ __align__(16) double Bs[GK][GP];   // [k][col]
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int64_t r0 = (int64_t)blockIdx.y * GT, c0 = (int64_t)blockIdx.x * GT;
+  double acc[8][8];
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int a = 0; a < 8; ++a)
 #pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
-  for (int kh = 0; kh < NB; kh += KH) {
-    for (int e = threadIdx.x; e < TM * KH; e += blockDim.x) {
-      const int rr = e / KH, kk = e % KH;
+    for (int b = 0; b < 8; ++b) acc[a][b] = 0.0;
+  // staging: a k-major operand ([row][k] in memory) is read as 16-byte k pairs,
+  // eight threads per row; a row-major one ([k][col]) as 16-byte column pairs
+  for (int k0 = 0; k0 < NB; k0 += GK) {
+#pragma unroll
+    for (int rep = 0; rep < 4; ++rep) {
+      const int e = rep * 256 + tid, rr = e >> 3, kp = (e & 7) * 2;
       const int64_t r = r0 + rr;
-      As[kk][rr] = r < m ? Ap[r * lda + kh + kk] : 0.0;
+      double2 v = make_double2(0.0, 0.0);
+      if (r < m) {
+        const double* src = Ap + r * lda + k0 + kp;
+        if (vec_a) v = *reinterpret_cast<const double2*>(src);
+        else v = make_double2(src[0], src[1]);
+      }
+      As[kp][rr] = v.x;
+      As[kp + 1][rr] = v.y;
     }
-    for (int e = threadIdx.x; e < TN * KH; e += blockDim.x) {
-      if (BT) {
-        const int cc = e / KH, kk = e % KH;
+    if (BT) {
+#pragma unroll
+      for (int rep = 0; rep < 4; ++rep) {
+        const int e = rep * 256 + tid, cc = e >> 3, kp = (e & 7) * 2;
         const int64_t c = c0 + cc;
-        Bs[kk][cc] = c < n ? Bp[c * ldb + kh + kk] : 0.0;
-      } else {
-        const int kk = e / TN, cc = e % TN;
-        const int64_t c = c0 + cc;
-        Bs[kk][cc] = c < n ? Bp[(int64_t)(kh + kk) * ldb + c] : 0.0;
+        double2 v = make_double2(0.0, 0.0);
+        if (c < n) {
+          const double* src = Bp + c * ldb + k0 + kp;
+          if (vec_b) v = *reinterpret_cast<const double2*>(src);
+          else v = make_double2(src[0], src[1]);
+        }
+        Bs[kp][cc] = v.x;
+        Bs[kp + 1][cc] = v.y;
+      }
+    } else {
+#pragma unroll
+      for (int rep = 0; rep < 4; ++rep) {
+        const int e = rep * 256 + tid, kk = e >> 6, cp = (e & 63) * 2;
+        const int64_t c = c0 + cp;
+        const double* src = Bp + (int64_t)(k0 + kk) * ldb + c;
+        double2 v;
+        v.x = c < n ? src[0] : 0.0;
+        v.y = c + 1 < n ? src[1] : 0.0;
+        *reinterpret_cast<double2*>(&Bs[kk][cp]) = v;
       }
     }
     __syncthreads();
-#pragma unroll 8
-    for (int kk = 0; kk < KH; ++kk) {
-      double av[4], bv[4];
 #pragma unroll
-      for (int a = 0; a < 4; ++a) av[a] = As[kk][ty * 4 + a];
+    for (int kk = 0; kk < GK; ++kk) {
+      double av[8], bv[8];
+      const double2 a0 = *reinterpret_cast<const double2*>(&As[kk][ty * 4]);
+      const double2 a1 = *reinterpret_cast<const double2*>(&As[kk][ty * 4 + 2]);
+      const double2 a2 = *reinterpret_cast<const double2*>(&As[kk][64 + ty * 4]);
+      const double2 a3 = *reinterpret_cast<const double2*>(&As[kk][64 + ty * 4 + 2]);
+      const double2 b0 = *reinterpret_cast<const double2*>(&Bs[kk][tx * 4]);
+      const double2 b1 = *reinterpret_cast<const double2*>(&Bs[kk][tx * 4 + 2]);
+      const double2 b2 = *reinterpret_cast<const double2*>(&Bs[kk][64 + tx * 4]);
+      const double2 b3 = *reinterpret_cast<const double2*>(&Bs[kk][64 + tx * 4 + 2]);
+      av[0] = a0.x; av[1] = a0.y; av[2] = a1.x; av[3] = a1.y; av[4] = a2.x; av[5] = a2.y; av[6] = a3.x; av[7] = a3.y;
+      bv[0] = b0.x; bv[1] = b0.y; bv[2] = b1.x; bv[3] = b1.y; bv[4] = b2.x; bv[5] = b2.y; bv[6] = b3.x; bv[7] = b3.y;
 #pragma unroll
-      for (int b = 0; b < 4; ++b) bv[b] = Bs[kk][tx * 4 + b];
+      for (int a = 0; a < 8; ++a)
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] += av[a] * bv[b];
+        for (int b = 0; b < 8; ++b) acc[a][b] = fma(av[a], bv[b], acc[a][b]);
     }
     __syncthreads();
   }
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    const int64_t r = r0 + ty * 4 + a;
+  for (int a = 0; a < 8; ++a) {
+    const int64_t r = r0 + (a < 4 ? ty * 4 + a : 64 + ty * 4 + a - 4);
     if (r >= m) continue;
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int64_t c = c0 + tx * 4 + b;
+    for (int b = 0; b < 8; ++b) {
+      const int64_t c = c0 + (b < 4 ? tx * 4 + b : 64 + tx * 4 + b - 4);
       if (c < n) C[r * ldc + c] -= acc[a][b];
     }
   }
@@ -340,8 +375,10 @@ __global__ void identity_kernel(double* __restrict__ Mx, int64_t d) {
 
 // Block row r0 of the inverse of the lower factor L: Mx[r0:r0+kb][c] =
 // L_rr^-1 Mx[r0:r0+kb][c] (forward substitution), one thread per column
-__global__ void __launch_bounds__(128) trtri_rows_kernel(const double* __restrict__ L, double* __restrict__ Mx,
-                                                         int64_t d, int64_t r0, int kb) {
+template <bool FULL>
+__global__ void __launch_bounds__(64) trtri_rows_kernel(const double* __restrict__ L, double* __restrict__ Mx,
+                                                        int64_t d, int64_t r0, int kb) {
+  if (FULL) kb = NB;
   __shared__ double l[NB][NB + 1];
   for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
     const int r = e / NB, c = e % NB;
@@ -351,18 +388,25 @@ __global__ void __launch_bounds__(128) trtri_rows_kernel(const double* __restric
   const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (c >= r0 + kb) return;
   double x[NB];
-#pragma unroll
-  for (int r = 0; r < NB; ++r) x[r] = r < kb ? Mx[(r0 + r) * d + c] : 0.0;
+  const double* src = Mx + r0 * d + c;
 #pragma unroll
   for (int r = 0; r < NB; ++r) {
-    double v = x[r];
-#pragma unroll
-    for (int q = 0; q < r; ++q) v -= l[r][q] * x[q];
-    x[r] = v / l[r][r];
+    x[r] = r < kb ? *src : 0.0;
+    src += d;
   }
 #pragma unroll
-  for (int r = 0; r < NB; ++r)
-    if (r < kb) Mx[(r0 + r) * d + c] = x[r];
+  for (int r = 0; r < NB; ++r) {
+    double p[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+    for (int q = 0; q < r; ++q) p[q & 3] = fma(l[r][q], x[q], p[q & 3]);
+    x[r] = (x[r] - ((p[0] + p[1]) + (p[2] + p[3]))) / l[r][r];
+  }
+  double* dst = Mx + r0 * d + c;
+#pragma unroll
+  for (int r = 0; r < NB; ++r) {
+    if (r < kb) *dst = x[r];
+    dst += d;
+  }
 }
 
 // U[j][k] = Mx[d-1-j][d-1-k]: element e swaps with element d*d - 1 - e
@@ -376,16 +420,28 @@ __global__ void reverse_kernel(double* __restrict__ Mx, int64_t d) {
   }
 }
 
-// diag(H^-1)[j] = sum_{k <= j} U[k][j]^2, rows in order
-__global__ void colnorm_kernel(const double* __restrict__ U, int64_t d, double* __restrict__ out) {
-  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= d) return;
+// diag(H^-1)[j] = sum_{k <= j} U[k][j]^2: a CTA takes 32 columns, its eight
+// row phases sum rows k = phase mod 8 in order, then the phases are added in
+// order (deterministic)
+__global__ void __launch_bounds__(256) colnorm_kernel(const double* __restrict__ U, int64_t d,
+                                                      double* __restrict__ out) {
+  __shared__ double part[8][33];
+  const int tx = threadIdx.x & 31, ph = threadIdx.x >> 5;
+  const int64_t j = (int64_t)blockIdx.x * 32 + tx;
   double s = 0.0;
-  for (int64_t k = 0; k <= j; ++k) {
-    const double u = U[k * d + j];
-    s += u * u;
+  if (j < d)
+    for (int64_t k = ph; k <= j; k += 8) {
+      const double u = U[k * d + j];
+      s = fma(u, u, s);
+    }
+  part[ph][tx] = s;
+  __syncthreads();
+  if (ph == 0 && j < d) {
+    double t = 0.0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) t += part[q][tx];
+    out[j] = t;
   }
-  out[j] = s;
 }
 
 // ============================================================================
@@ -576,6 +632,10 @@ cudaError_t launch_gram(const uint16_t* X, int64_t s, int64_t d, float* H, int a
   return cudaGetLastError();
 }
 
+// 16-byte loads of a k-major operand need an even leading dimension and an
+// aligned base
+int vec16(const double* p, int64_t ld) { return (ld % 2 == 0 && (reinterpret_cast<uintptr_t>(p) & 15u) == 0) ? 1 : 0; }
+
 size_t inverse_factor_workspace(int64_t d) { return (size_t)d * (size_t)d * sizeof(double) + 256; }
 
 cudaError_t launch_inverse_factor(const float* H, int64_t d, double damp, double* U, double* hinv_diag,
@@ -594,11 +654,11 @@ cudaError_t launch_inverse_factor(const float* H, int64_t d, double damp, double
     potrf_diag_kernel<<<1, 256, 0, st>>>(A, d, k0, kb, check);
     const int64_t rest = d - k0 - kb;
     if (rest > 0) {
-      trsm_panel_kernel<<<(unsigned)cdiv(rest, 128), 128, 0, st>>>(A, d, k0);
+      trsm_panel_kernel<<<(unsigned)cdiv(rest, 64), 64, 0, st>>>(A, d, k0);
       const double* panel = A + (k0 + NB) * d + k0;
-      dim3 grid((unsigned)cdiv(rest, 64), (unsigned)cdiv(rest, 64));
+      dim3 grid((unsigned)cdiv(rest, GT), (unsigned)cdiv(rest, GT));
       gemm_sub_f64_kernel<true, true><<<grid, 256, 0, st>>>(panel, d, panel, d, A + (k0 + NB) * d + k0 + NB, d, rest,
-                                                            rest);
+                                                            rest, vec16(panel, d), vec16(panel, d));
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -607,18 +667,20 @@ cudaError_t launch_inverse_factor(const float* H, int64_t d, double damp, double
   identity_kernel<<<eg, 256, 0, st>>>(U, d);
   for (int64_t r0 = 0; r0 < d; r0 += NB) {
     const int kb = (int)(d - r0 < NB ? d - r0 : NB);
-    trtri_rows_kernel<<<(unsigned)cdiv(r0 + kb, 128), 128, 0, st>>>(A, U, d, r0, kb);
+    if (kb == NB) trtri_rows_kernel<true><<<(unsigned)cdiv(r0 + kb, 64), 64, 0, st>>>(A, U, d, r0, kb);
+    else trtri_rows_kernel<false><<<(unsigned)cdiv(r0 + kb, 64), 64, 0, st>>>(A, U, d, r0, kb);
     const int64_t rest = d - r0 - kb;
     if (rest > 0) {
-      dim3 grid((unsigned)cdiv(r0 + kb, 64), (unsigned)cdiv(rest, 64));
-      gemm_sub_f64_kernel<false, false><<<grid, 256, 0, st>>>(A + (r0 + NB) * d + r0, d, U + r0 * d, d,
-                                                              U + (r0 + NB) * d, d, rest, r0 + kb);
+      dim3 grid((unsigned)cdiv(r0 + kb, GT), (unsigned)cdiv(rest, GT));
+      const double* Ab = A + (r0 + NB) * d + r0;
+      gemm_sub_f64_kernel<false, false><<<grid, 256, 0, st>>>(Ab, d, U + r0 * d, d, U + (r0 + NB) * d, d, rest,
+                                                              r0 + kb, vec16(Ab, d), 0);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   reverse_kernel<<<(unsigned)((dd / 2 + 255) / 256 > 0 ? (dd / 2 + 255) / 256 : 1), 256, 0, st>>>(U, d);
-  colnorm_kernel<<<(unsigned)cdiv(d, 128), 128, 0, st>>>(U, d, hinv_diag);
+  colnorm_kernel<<<(unsigned)cdiv(d, 32), 256, 0, st>>>(U, d, hinv_diag);
   return cudaGetLastError();
 }
 
@@ -636,13 +698,13 @@ cudaError_t launch_lloyd(const float* theta, const double* hinv_diag, int bits, 
 }
 
 size_t sketch_round_workspace(int64_t n, int64_t d) {
-  return ((size_t)n * (size_t)d + (size_t)n * NB) * sizeof(double) + 256;
+  return (((size_t)n * (size_t)d + 1) / 2 * 2 + (size_t)n * NB) * sizeof(double) + 256;
 }
 
 cudaError_t launch_sketch_round(const float* theta, const double* U, const uint16_t* lut, int bits, int gpr, int64_t n,
                                 int64_t d, uint8_t* idx, void* workspace, unsigned int* check, cudaStream_t st) {
   double* W = static_cast<double*>(workspace);   // [n][d] values being mapped
-  double* E = W + n * d;                         // [n][NB] errors of the current block
+  double* E = W + (n * d + 1) / 2 * 2;           // [n][NB] errors of the current block (16-byte aligned)
   const int64_t gs = d / gpr;
   const int k = 1 << bits;
   round_init_kernel<<<(unsigned)(num_sms() * 8), 256, 0, st>>>(theta, n * d, W);
@@ -654,8 +716,9 @@ cudaError_t launch_sketch_round(const float* theta, const double* U, const uint1
     round_block_kernel<<<rgrid, kRoundWarps * 32, 0, st>>>(W, U, lut, n, d, gs, gpr, k, j0, kb, E, idx, check);
     const int64_t rest = d - j0 - kb;
     if (rest > 0) {
-      dim3 grid((unsigned)cdiv(rest, 64), (unsigned)cdiv(n, 64));
-      gemm_sub_f64_kernel<false, false><<<grid, 256, 0, st>>>(E, NB, U + j0 * d + j0 + NB, d, W + j0 + NB, d, n, rest);
+      dim3 grid((unsigned)cdiv(rest, GT), (unsigned)cdiv(n, GT));
+      gemm_sub_f64_kernel<false, false><<<grid, 256, 0, st>>>(E, NB, U + j0 * d + j0 + NB, d, W + j0 + NB, d, n, rest,
+                                                              vec16(E, NB), 0);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

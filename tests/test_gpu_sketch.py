@@ -113,7 +113,7 @@ def _gram_f32(seed, d, s=None):
     return oracle.gram(x).astype(np.float32)
 
 
-@pytest.mark.parametrize("d", [1, 40, 64, 200, 1024])
+@pytest.mark.parametrize("d", [1, 40, 64, 65, 200, 331, 1024])
 def test_inverse_factor_matches_oracle(d):
     h32 = _gram_f32(60010 + d, d)
     U, hd = _sk().inverse_factor(torch.from_numpy(h32).cuda(), 0.01)
@@ -217,7 +217,7 @@ def test_lloyd_full_size_sampled():
 # ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("bits,n,d,gpr", [(2, 5, 32, 1), (4, 40, 200, 5), (3, 17, 256, 2), (4, 64, 1024, 8),
-                                          (2, 33, 520, 4)])
+                                          (2, 33, 520, 4), (3, 7, 195, 3), (4, 129, 65, 1)])
 def test_sketch_round_matches_oracle(bits, n, d, gpr):
     rng = synth.rng_for(60500 + n + d)
     theta = (rng.standard_normal((n, d)) * 0.02).astype(np.float32)
