@@ -42,7 +42,10 @@ __host__ __device__ constexpr int ceil_div(int64_t a, int64_t b) { return (int)(
 namespace dx {
 constexpr int N = 256;          // tokens per tile
 constexpr int KS = 64;          // weight rows (K) per pipeline step
-constexpr int S = 4;            // stages
+// two stages, so that two CTAs share an SM (the dequantising warps of one
+// overlap the other's MMAs and epilogue): measured 21 % faster than one CTA
+// with four stages on the 7B gate_proj at 8192 tokens
+constexpr int S = 2;
 constexpr int B_BYTES = N * 128;             // dY tile: N rows x 64 bf16
 constexpr int A_BYTES = 2 * 8 * 1024;        // two 64-column MN atoms x 8 K-groups
 constexpr int STAGE = B_BYTES + A_BYTES;
@@ -69,7 +72,7 @@ struct DxArgs {
 };
 
 template <int BITS>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 dx_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, DxArgs a) {
   using namespace dx;
   extern __shared__ uint8_t smem_raw[];
