@@ -270,7 +270,8 @@ __global__ void __launch_bounds__(64) trsm_panel_kernel(double* __restrict__ A, 
   for (int c = 0; c < NB; ++c) row[c] = x[c];
 }
 
-// C[m][n] -= A[m][NB] * B, with B(k, c) = B[c][k] (BT) or B[k][c].  128 x 128
+// C[m][n] -= A[m][K] * B, with B(k, c) = B[c][k] (BT) or B[k][c], K a multiple
+// of 16 (64 or 128: the rank of one blocked update).  128 x 128
 // output tiles, 8 x 8 per thread (rows ty*4 + {0..3} and 64 + ty*4 + {0..3},
 // likewise the columns), K in chunks of 16 staged k-major in shared memory:
 // per k a thread loads 8 + 8 doubles for 64 FMAs, which keeps the float64
@@ -282,7 +283,7 @@ template <bool BT, bool LOWER>
 __global__ void __launch_bounds__(256, 1) gemm_sub_f64_kernel(const double* __restrict__ Ap, int64_t lda,
                                                               const double* __restrict__ Bp, int64_t ldb,
                                                               double* __restrict__ C, int64_t ldc, int64_t m,
-                                                              int64_t n, int vec_a, int vec_b) {
+                                                              int64_t n, int K, int vec_a, int vec_b) {
   if (LOWER && blockIdx.x > blockIdx.y) return;
   __shared__ __align__(16) double As[GK][GP];   // [k][row]
   __shared__ __align__(16) double Bs[GK][GP];   // [k][col]
@@ -295,7 +296,7 @@ __global__ void __launch_bounds__(256, 1) gemm_sub_f64_kernel(const double* __re
     for (int b = 0; b < 8; ++b) acc[a][b] = 0.0;
   // staging: a k-major operand ([row][k] in memory) is read as 16-byte k pairs,
   // eight threads per row; a row-major one ([k][col]) as 16-byte column pairs
-  for (int k0 = 0; k0 < NB; k0 += GK) {
+  for (int k0 = 0; k0 < K; k0 += GK) {
 #pragma unroll
     for (int rep = 0; rep < 4; ++rep) {
       const int e = rep * 256 + tid, rr = e >> 3, kp = (e & 7) * 2;
@@ -556,6 +557,8 @@ lloyd_kernel(const float* __restrict__ theta, const double* __restrict__ hinv, i
 // ============================================================================
 
 constexpr int kRoundWarps = 16;   // rows per CTA, one warp each
+constexpr int RB = 128;           // columns per mapping block (the rank of its lazy update)
+constexpr int RQ = RB / 32;       // columns per lane
 
 __global__ void round_init_kernel(const float* __restrict__ theta, int64_t count, double* __restrict__ W) {
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < count; e += (int64_t)gridDim.x * blockDim.x)
@@ -565,25 +568,31 @@ __global__ void round_init_kernel(const float* __restrict__ theta, int64_t count
 // Columns [j0, j0 + kb) of every row, in order: the nearest fp16 centroid of
 // the current value (float32 midpoints, ties to the lower centroid), the
 // error e = (w_j - q_j) / U_jj, and w_c -= e U_jc for the block's later
-// columns c.  A lane holds columns j0 + lane and j0 + 32 + lane of its row.
-// The errors go to E [n][NB] for the GEMM that updates the later blocks.
+// columns c.  A lane holds columns j0 + 32 q + lane (q < 4) of its row; the
+// block of U sits in shared memory ([RB][RB] doubles, dynamic).  The errors
+// go to E [n][RB] for the GEMM that updates the later blocks.
 __global__ void __launch_bounds__(kRoundWarps * 32)
 round_block_kernel(double* __restrict__ W, const double* __restrict__ U, const uint16_t* __restrict__ lut, int64_t n,
                    int64_t d, int64_t gs, int gpr, int k, int64_t j0, int kb, double* __restrict__ E,
                    uint8_t* __restrict__ idx, unsigned int* check) {
-  __shared__ double ub[NB][NB + 1];   // U[j0 + a][j0 + b]
-  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
-    const int a = e / NB, b = e % NB;
-    ub[a][b] = (a < kb && b < kb) ? U[(j0 + a) * d + j0 + b] : 0.0;
+  extern __shared__ __align__(16) double ub[];   // U[j0 + a][j0 + b] at a * RB + b
+  for (int e = threadIdx.x; e < RB * RB; e += blockDim.x) {
+    const int a = e / RB, b = e % RB;
+    ub[e] = (a < kb && b < kb) ? U[(j0 + a) * d + j0 + b] : 0.0;
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t i = (int64_t)blockIdx.x * kRoundWarps + warp;
   if (i >= n) return;
   double* wrow = W + i * d + j0;
-  double w0 = lane < kb ? wrow[lane] : 0.0, w1 = 32 + lane < kb ? wrow[32 + lane] : 0.0;
-  double e0 = 0.0, e1 = 0.0;
-  int c0 = 0, c1 = 0;
+  double w[RQ], e_own[RQ];
+  int c_own[RQ];
+#pragma unroll
+  for (int q = 0; q < RQ; ++q) {
+    w[q] = 32 * q + lane < kb ? wrow[32 * q + lane] : 0.0;
+    e_own[q] = 0.0;
+    c_own[q] = 0;
+  }
   int cur_g = -1;
   float cent = 0.f, mid = 0.f;
   for (int jj = 0; jj < kb; ++jj) {
@@ -596,21 +605,34 @@ round_block_kernel(double* __restrict__ W, const double* __restrict__ U, const u
       mid = midpoint(cent, next);
       if (lane < k - 1 && next < cent) atomicOr(check, SK_CHECK_LUT_ORDER);
     }
-    const double th = __shfl_sync(0xffffffffu, jj < 32 ? w0 : w1, jj & 31);
+    const int qj = jj >> 5;
+    double mine = w[0];
+#pragma unroll
+    for (int q = 1; q < RQ; ++q)
+      if (q == qj) mine = w[q];
+    const double th = __shfl_sync(0xffffffffu, mine, jj & 31);
     const int c = __popc(__ballot_sync(0xffffffffu, lane < k - 1 && th > (double)mid));
-    const double q = (double)__shfl_sync(0xffffffffu, cent, c);
-    const double e = __ddiv_rn(__dsub_rn(th, q), ub[jj][jj]);
-    if (lane > jj && lane < kb) w0 = __dsub_rn(w0, __dmul_rn(e, ub[jj][lane]));
-    if (32 + lane > jj && 32 + lane < kb) w1 = __dsub_rn(w1, __dmul_rn(e, ub[jj][32 + lane]));
+    const double qv = (double)__shfl_sync(0xffffffffu, cent, c);
+    const double e = __ddiv_rn(__dsub_rn(th, qv), ub[jj * RB + jj]);
+    const double* urow = ub + jj * RB;
+#pragma unroll
+    for (int q = 0; q < RQ; ++q) {
+      const int col = 32 * q + lane;
+      if (col > jj && col < kb) w[q] = __dsub_rn(w[q], __dmul_rn(e, urow[col]));
+    }
     if (lane == (jj & 31)) {
-      if (jj < 32) { e0 = e; c0 = c; } else { e1 = e; c1 = c; }
+#pragma unroll
+      for (int q = 0; q < RQ; ++q)
+        if (q == qj) { e_own[q] = e; c_own[q] = c; }
     }
   }
-  double* erow = E + i * NB;
-  erow[lane] = lane < kb ? e0 : 0.0;
-  erow[32 + lane] = 32 + lane < kb ? e1 : 0.0;
-  if (lane < kb) idx[i * d + j0 + lane] = (uint8_t)c0;
-  if (32 + lane < kb) idx[i * d + j0 + 32 + lane] = (uint8_t)c1;
+  double* erow = E + i * RB;
+#pragma unroll
+  for (int q = 0; q < RQ; ++q) {
+    const int col = 32 * q + lane;
+    erow[col] = col < kb ? e_own[q] : 0.0;
+    if (col < kb) idx[i * d + j0 + col] = (uint8_t)c_own[q];
+  }
 }
 
 }  // namespace
@@ -648,33 +670,65 @@ cudaError_t launch_inverse_factor(const float* H, int64_t d, double damp, double
   reverse_damp_kernel<<<eg, 256, 0, st>>>(H, d, lam, A);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  // blocked Cholesky (lower) of A
-  for (int64_t k0 = 0; k0 < d; k0 += NB) {
-    const int kb = (int)(d - k0 < NB ? d - k0 : NB);
-    potrf_diag_kernel<<<1, 256, 0, st>>>(A, d, k0, kb, check);
-    const int64_t rest = d - k0 - kb;
+  // blocked Cholesky (lower) of A in super-blocks of two 64-column blocks:
+  // inside a super-block the first block's panel updates only the second
+  // block's columns; the rest of the trailing matrix takes one rank-128 update
+  for (int64_t k0 = 0; k0 < d; k0 += 2 * NB) {
+    for (int h = 0; h < 2; ++h) {
+      const int64_t kk = k0 + h * NB;
+      if (kk >= d) break;
+      const int kb = (int)(d - kk < NB ? d - kk : NB);
+      potrf_diag_kernel<<<1, 256, 0, st>>>(A, d, kk, kb, check);
+      const int64_t rest = d - kk - kb;
+      if (rest > 0) trsm_panel_kernel<<<(unsigned)cdiv(rest, 64), 64, 0, st>>>(A, d, kk);
+      if (h == 0 && rest > 0) {
+        const int64_t n2 = rest < NB ? rest : NB;      // columns of the second block
+        const double* panel = A + (kk + NB) * d + kk;
+        dim3 grid((unsigned)cdiv(n2, GT), (unsigned)cdiv(rest, GT));
+        gemm_sub_f64_kernel<true, false><<<grid, 256, 0, st>>>(panel, d, panel, d, A + (kk + NB) * d + kk + NB, d,
+                                                               rest, n2, NB, vec16(panel, d), vec16(panel, d));
+      }
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    const int64_t kw = d - k0 < 2 * NB ? d - k0 : 2 * NB;
+    const int64_t rest = d - k0 - kw;
     if (rest > 0) {
-      trsm_panel_kernel<<<(unsigned)cdiv(rest, 64), 64, 0, st>>>(A, d, k0);
-      const double* panel = A + (k0 + NB) * d + k0;
+      const double* panel = A + (k0 + kw) * d + k0;
       dim3 grid((unsigned)cdiv(rest, GT), (unsigned)cdiv(rest, GT));
-      gemm_sub_f64_kernel<true, true><<<grid, 256, 0, st>>>(panel, d, panel, d, A + (k0 + NB) * d + k0 + NB, d, rest,
-                                                            rest, vec16(panel, d), vec16(panel, d));
+      gemm_sub_f64_kernel<true, true><<<grid, 256, 0, st>>>(panel, d, panel, d, A + (k0 + kw) * d + k0 + kw, d, rest,
+                                                            rest, (int)kw, vec16(panel, d), vec16(panel, d));
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  // U buffer: inverse of the lower factor by blocked forward substitution
+  // U buffer: inverse of the lower factor by blocked forward substitution,
+  // in the same super-blocks
   identity_kernel<<<eg, 256, 0, st>>>(U, d);
-  for (int64_t r0 = 0; r0 < d; r0 += NB) {
-    const int kb = (int)(d - r0 < NB ? d - r0 : NB);
-    if (kb == NB) trtri_rows_kernel<true><<<(unsigned)cdiv(r0 + kb, 64), 64, 0, st>>>(A, U, d, r0, kb);
-    else trtri_rows_kernel<false><<<(unsigned)cdiv(r0 + kb, 64), 64, 0, st>>>(A, U, d, r0, kb);
-    const int64_t rest = d - r0 - kb;
+  for (int64_t r0 = 0; r0 < d; r0 += 2 * NB) {
+    for (int h = 0; h < 2; ++h) {
+      const int64_t rr = r0 + h * NB;
+      if (rr >= d) break;
+      const int kb = (int)(d - rr < NB ? d - rr : NB);
+      if (kb == NB) trtri_rows_kernel<true><<<(unsigned)cdiv(rr + kb, 64), 64, 0, st>>>(A, U, d, rr, kb);
+      else trtri_rows_kernel<false><<<(unsigned)cdiv(rr + kb, 64), 64, 0, st>>>(A, U, d, rr, kb);
+      const int64_t rows2 = d - rr - kb < NB ? d - rr - kb : NB;   // rows of the second block
+      if (h == 0 && rows2 > 0) {
+        const double* Ab = A + (rr + NB) * d + rr;
+        dim3 grid((unsigned)cdiv(rr + kb, GT), (unsigned)cdiv(rows2, GT));
+        gemm_sub_f64_kernel<false, false><<<grid, 256, 0, st>>>(Ab, d, U + rr * d, d, U + (rr + NB) * d, d, rows2,
+                                                                rr + kb, NB, vec16(Ab, d), 0);
+      }
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    const int64_t kw = d - r0 < 2 * NB ? d - r0 : 2 * NB;
+    const int64_t rest = d - r0 - kw;
     if (rest > 0) {
-      dim3 grid((unsigned)cdiv(r0 + kb, GT), (unsigned)cdiv(rest, GT));
-      const double* Ab = A + (r0 + NB) * d + r0;
-      gemm_sub_f64_kernel<false, false><<<grid, 256, 0, st>>>(Ab, d, U + r0 * d, d, U + (r0 + NB) * d, d, rest,
-                                                              r0 + kb, vec16(Ab, d), 0);
+      const double* Ab = A + (r0 + kw) * d + r0;
+      dim3 grid((unsigned)cdiv(r0 + kw, GT), (unsigned)cdiv(rest, GT));
+      gemm_sub_f64_kernel<false, false><<<grid, 256, 0, st>>>(Ab, d, U + r0 * d, d, U + (r0 + kw) * d, d, rest,
+                                                              r0 + kw, (int)kw, vec16(Ab, d), 0);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -698,27 +752,31 @@ cudaError_t launch_lloyd(const float* theta, const double* hinv_diag, int bits, 
 }
 
 size_t sketch_round_workspace(int64_t n, int64_t d) {
-  return (((size_t)n * (size_t)d + 1) / 2 * 2 + (size_t)n * NB) * sizeof(double) + 256;
+  return (((size_t)n * (size_t)d + 1) / 2 * 2 + (size_t)n * RB) * sizeof(double) + 256;
 }
 
 cudaError_t launch_sketch_round(const float* theta, const double* U, const uint16_t* lut, int bits, int gpr, int64_t n,
                                 int64_t d, uint8_t* idx, void* workspace, unsigned int* check, cudaStream_t st) {
   double* W = static_cast<double*>(workspace);   // [n][d] values being mapped
-  double* E = W + (n * d + 1) / 2 * 2;           // [n][NB] errors of the current block (16-byte aligned)
+  double* E = W + (n * d + 1) / 2 * 2;           // [n][RB] errors of the current block (16-byte aligned)
   const int64_t gs = d / gpr;
   const int k = 1 << bits;
   round_init_kernel<<<(unsigned)(num_sms() * 8), 256, 0, st>>>(theta, n * d, W);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = cudaFuncSetAttribute(round_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       RB * RB * (int)sizeof(double));
+  if (e != cudaSuccess) return e;
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const unsigned rgrid = (unsigned)cdiv(n, kRoundWarps);
-  for (int64_t j0 = 0; j0 < d; j0 += NB) {
-    const int kb = (int)(d - j0 < NB ? d - j0 : NB);
-    round_block_kernel<<<rgrid, kRoundWarps * 32, 0, st>>>(W, U, lut, n, d, gs, gpr, k, j0, kb, E, idx, check);
+  for (int64_t j0 = 0; j0 < d; j0 += RB) {
+    const int kb = (int)(d - j0 < RB ? d - j0 : RB);
+    round_block_kernel<<<rgrid, kRoundWarps * 32, RB * RB * sizeof(double), st>>>(W, U, lut, n, d, gs, gpr, k, j0, kb,
+                                                                                  E, idx, check);
     const int64_t rest = d - j0 - kb;
     if (rest > 0) {
       dim3 grid((unsigned)cdiv(rest, GT), (unsigned)cdiv(n, GT));
-      gemm_sub_f64_kernel<false, false><<<grid, 256, 0, st>>>(E, NB, U + j0 * d + j0 + NB, d, W + j0 + NB, d, n, rest,
-                                                              vec16(E, NB), 0);
+      gemm_sub_f64_kernel<false, false><<<grid, 256, 0, st>>>(E, RB, U + j0 * d + j0 + RB, d, W + j0 + RB, d, n, rest,
+                                                              RB, vec16(E, RB), 0);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
