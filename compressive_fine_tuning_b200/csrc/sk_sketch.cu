@@ -285,8 +285,10 @@ __global__ void __launch_bounds__(256, 1) gemm_sub_f64_kernel(const double* __re
                                                               double* __restrict__ C, int64_t ldc, int64_t m,
                                                               int64_t n, int K, int vec_a, int vec_b) {
   if (LOWER && blockIdx.x > blockIdx.y) return;
-  __shared__ __align__(16) double As[GK][GP];   // [k][row]
-  __shared__ __align__(16) double Bs[GK][GP];   // [k][col]
+  // two buffers of [A: GK][GP] + [B: GK][GP]; the next K chunk is loaded into
+  // registers while the current one is multiplied, then stored to the other
+  // buffer, so global latency hides behind the FMAs (one barrier per chunk)
+  extern __shared__ __align__(16) double gsm[];
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const int64_t r0 = (int64_t)blockIdx.y * GT, c0 = (int64_t)blockIdx.x * GT;
   double acc[8][8];
@@ -294,60 +296,82 @@ __global__ void __launch_bounds__(256, 1) gemm_sub_f64_kernel(const double* __re
   for (int a = 0; a < 8; ++a)
 #pragma unroll
     for (int b = 0; b < 8; ++b) acc[a][b] = 0.0;
+  double2 pa[4], pb[4];
   // staging: a k-major operand ([row][k] in memory) is read as 16-byte k pairs,
   // eight threads per row; a row-major one ([k][col]) as 16-byte column pairs
-  for (int k0 = 0; k0 < K; k0 += GK) {
+  auto fetch = [&](int k0) {
 #pragma unroll
     for (int rep = 0; rep < 4; ++rep) {
       const int e = rep * 256 + tid, rr = e >> 3, kp = (e & 7) * 2;
       const int64_t r = r0 + rr;
-      double2 v = make_double2(0.0, 0.0);
+      pa[rep] = make_double2(0.0, 0.0);
       if (r < m) {
         const double* src = Ap + r * lda + k0 + kp;
-        if (vec_a) v = *reinterpret_cast<const double2*>(src);
-        else v = make_double2(src[0], src[1]);
+        pa[rep] = vec_a ? *reinterpret_cast<const double2*>(src) : make_double2(src[0], src[1]);
       }
-      As[kp][rr] = v.x;
-      As[kp + 1][rr] = v.y;
     }
-    if (BT) {
 #pragma unroll
-      for (int rep = 0; rep < 4; ++rep) {
-        const int e = rep * 256 + tid, cc = e >> 3, kp = (e & 7) * 2;
+    for (int rep = 0; rep < 4; ++rep) {
+      const int e = rep * 256 + tid;
+      if (BT) {
+        const int cc = e >> 3, kp = (e & 7) * 2;
         const int64_t c = c0 + cc;
-        double2 v = make_double2(0.0, 0.0);
+        pb[rep] = make_double2(0.0, 0.0);
         if (c < n) {
           const double* src = Bp + c * ldb + k0 + kp;
-          if (vec_b) v = *reinterpret_cast<const double2*>(src);
-          else v = make_double2(src[0], src[1]);
+          pb[rep] = vec_b ? *reinterpret_cast<const double2*>(src) : make_double2(src[0], src[1]);
         }
-        Bs[kp][cc] = v.x;
-        Bs[kp + 1][cc] = v.y;
-      }
-    } else {
-#pragma unroll
-      for (int rep = 0; rep < 4; ++rep) {
-        const int e = rep * 256 + tid, kk = e >> 6, cp = (e & 63) * 2;
+      } else {
+        const int kk = e >> 6, cp = (e & 63) * 2;
         const int64_t c = c0 + cp;
         const double* src = Bp + (int64_t)(k0 + kk) * ldb + c;
-        double2 v;
-        v.x = c < n ? src[0] : 0.0;
-        v.y = c + 1 < n ? src[1] : 0.0;
-        *reinterpret_cast<double2*>(&Bs[kk][cp]) = v;
+        pb[rep].x = c < n ? src[0] : 0.0;
+        pb[rep].y = c + 1 < n ? src[1] : 0.0;
       }
     }
-    __syncthreads();
+  };
+  auto stash = [&](int buf) {
+    double* As = gsm + buf * 2 * GK * GP;   // [k][row]
+    double* Bs = As + GK * GP;              // [k][col]
+#pragma unroll
+    for (int rep = 0; rep < 4; ++rep) {
+      const int e = rep * 256 + tid, rr = e >> 3, kp = (e & 7) * 2;
+      As[kp * GP + rr] = pa[rep].x;
+      As[(kp + 1) * GP + rr] = pa[rep].y;
+    }
+#pragma unroll
+    for (int rep = 0; rep < 4; ++rep) {
+      const int e = rep * 256 + tid;
+      if (BT) {
+        const int cc = e >> 3, kp = (e & 7) * 2;
+        Bs[kp * GP + cc] = pb[rep].x;
+        Bs[(kp + 1) * GP + cc] = pb[rep].y;
+      } else {
+        const int kk = e >> 6, cp = (e & 63) * 2;
+        *reinterpret_cast<double2*>(&Bs[kk * GP + cp]) = pb[rep];
+      }
+    }
+  };
+  fetch(0);
+  stash(0);
+  __syncthreads();
+  int buf = 0;
+  for (int k0 = 0; k0 < K; k0 += GK) {
+    const bool more = k0 + GK < K;
+    if (more) fetch(k0 + GK);
+    const double* As = gsm + buf * 2 * GK * GP;
+    const double* Bs = As + GK * GP;
 #pragma unroll
     for (int kk = 0; kk < GK; ++kk) {
       double av[8], bv[8];
-      const double2 a0 = *reinterpret_cast<const double2*>(&As[kk][ty * 4]);
-      const double2 a1 = *reinterpret_cast<const double2*>(&As[kk][ty * 4 + 2]);
-      const double2 a2 = *reinterpret_cast<const double2*>(&As[kk][64 + ty * 4]);
-      const double2 a3 = *reinterpret_cast<const double2*>(&As[kk][64 + ty * 4 + 2]);
-      const double2 b0 = *reinterpret_cast<const double2*>(&Bs[kk][tx * 4]);
-      const double2 b1 = *reinterpret_cast<const double2*>(&Bs[kk][tx * 4 + 2]);
-      const double2 b2 = *reinterpret_cast<const double2*>(&Bs[kk][64 + tx * 4]);
-      const double2 b3 = *reinterpret_cast<const double2*>(&Bs[kk][64 + tx * 4 + 2]);
+      const double2 a0 = *reinterpret_cast<const double2*>(&As[kk * GP + ty * 4]);
+      const double2 a1 = *reinterpret_cast<const double2*>(&As[kk * GP + ty * 4 + 2]);
+      const double2 a2 = *reinterpret_cast<const double2*>(&As[kk * GP + 64 + ty * 4]);
+      const double2 a3 = *reinterpret_cast<const double2*>(&As[kk * GP + 64 + ty * 4 + 2]);
+      const double2 b0 = *reinterpret_cast<const double2*>(&Bs[kk * GP + tx * 4]);
+      const double2 b1 = *reinterpret_cast<const double2*>(&Bs[kk * GP + tx * 4 + 2]);
+      const double2 b2 = *reinterpret_cast<const double2*>(&Bs[kk * GP + 64 + tx * 4]);
+      const double2 b3 = *reinterpret_cast<const double2*>(&Bs[kk * GP + 64 + tx * 4 + 2]);
       av[0] = a0.x; av[1] = a0.y; av[2] = a1.x; av[3] = a1.y; av[4] = a2.x; av[5] = a2.y; av[6] = a3.x; av[7] = a3.y;
       bv[0] = b0.x; bv[1] = b0.y; bv[2] = b1.x; bv[3] = b1.y; bv[4] = b2.x; bv[5] = b2.y; bv[6] = b3.x; bv[7] = b3.y;
 #pragma unroll
@@ -355,7 +379,9 @@ __global__ void __launch_bounds__(256, 1) gemm_sub_f64_kernel(const double* __re
 #pragma unroll
         for (int b = 0; b < 8; ++b) acc[a][b] = fma(av[a], bv[b], acc[a][b]);
     }
+    if (more) stash(buf ^ 1);
     __syncthreads();
+    buf ^= 1;
   }
 #pragma unroll
   for (int a = 0; a < 8; ++a) {
@@ -368,6 +394,8 @@ __global__ void __launch_bounds__(256, 1) gemm_sub_f64_kernel(const double* __re
     }
   }
 }
+
+constexpr int kGemmSmem = 2 * 2 * GK * GP * (int)sizeof(double);
 
 __global__ void identity_kernel(double* __restrict__ Mx, int64_t d) {
   const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -654,6 +682,18 @@ cudaError_t launch_gram(const uint16_t* X, int64_t s, int64_t d, float* H, int a
   return cudaGetLastError();
 }
 
+// the GEMM's double-buffered staging needs more than the default 48 KB of
+// dynamic shared memory
+cudaError_t gemm_smem_setup() {
+  cudaError_t e = cudaFuncSetAttribute(gemm_sub_f64_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kGemmSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gemm_sub_f64_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gemm_sub_f64_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+  return e;
+}
+
 // 16-byte loads of a k-major operand need an even leading dimension and an
 // aligned base
 int vec16(const double* p, int64_t ld) { return (ld % 2 == 0 && (reinterpret_cast<uintptr_t>(p) & 15u) == 0) ? 1 : 0; }
@@ -666,9 +706,11 @@ cudaError_t launch_inverse_factor(const float* H, int64_t d, double damp, double
   double* lam = A + d * d;
   const int64_t dd = d * d;
   const unsigned eg = (unsigned)((dd + 255) / 256);
+  cudaError_t e = gemm_smem_setup();
+  if (e != cudaSuccess) return e;
   damp_kernel<<<1, 1024, 0, st>>>(H, d, damp, lam);
   reverse_damp_kernel<<<eg, 256, 0, st>>>(H, d, lam, A);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // blocked Cholesky (lower) of A in super-blocks of two 64-column blocks:
   // inside a super-block the first block's panel updates only the second
@@ -685,7 +727,7 @@ cudaError_t launch_inverse_factor(const float* H, int64_t d, double damp, double
         const int64_t n2 = rest < NB ? rest : NB;      // columns of the second block
         const double* panel = A + (kk + NB) * d + kk;
         dim3 grid((unsigned)cdiv(n2, GT), (unsigned)cdiv(rest, GT));
-        gemm_sub_f64_kernel<true, false><<<grid, 256, 0, st>>>(panel, d, panel, d, A + (kk + NB) * d + kk + NB, d,
+        gemm_sub_f64_kernel<true, false><<<grid, 256, kGemmSmem, st>>>(panel, d, panel, d, A + (kk + NB) * d + kk + NB, d,
                                                                rest, n2, NB, vec16(panel, d), vec16(panel, d));
       }
       e = cudaGetLastError();
@@ -696,7 +738,7 @@ cudaError_t launch_inverse_factor(const float* H, int64_t d, double damp, double
     if (rest > 0) {
       const double* panel = A + (k0 + kw) * d + k0;
       dim3 grid((unsigned)cdiv(rest, GT), (unsigned)cdiv(rest, GT));
-      gemm_sub_f64_kernel<true, true><<<grid, 256, 0, st>>>(panel, d, panel, d, A + (k0 + kw) * d + k0 + kw, d, rest,
+      gemm_sub_f64_kernel<true, true><<<grid, 256, kGemmSmem, st>>>(panel, d, panel, d, A + (k0 + kw) * d + k0 + kw, d, rest,
                                                             rest, (int)kw, vec16(panel, d), vec16(panel, d));
     }
     e = cudaGetLastError();
@@ -716,7 +758,7 @@ cudaError_t launch_inverse_factor(const float* H, int64_t d, double damp, double
       if (h == 0 && rows2 > 0) {
         const double* Ab = A + (rr + NB) * d + rr;
         dim3 grid((unsigned)cdiv(rr + kb, GT), (unsigned)cdiv(rows2, GT));
-        gemm_sub_f64_kernel<false, false><<<grid, 256, 0, st>>>(Ab, d, U + rr * d, d, U + (rr + NB) * d, d, rows2,
+        gemm_sub_f64_kernel<false, false><<<grid, 256, kGemmSmem, st>>>(Ab, d, U + rr * d, d, U + (rr + NB) * d, d, rows2,
                                                                 rr + kb, NB, vec16(Ab, d), 0);
       }
       e = cudaGetLastError();
@@ -727,7 +769,7 @@ cudaError_t launch_inverse_factor(const float* H, int64_t d, double damp, double
     if (rest > 0) {
       const double* Ab = A + (r0 + kw) * d + r0;
       dim3 grid((unsigned)cdiv(r0 + kw, GT), (unsigned)cdiv(rest, GT));
-      gemm_sub_f64_kernel<false, false><<<grid, 256, 0, st>>>(Ab, d, U + r0 * d, d, U + (r0 + kw) * d, d, rest,
+      gemm_sub_f64_kernel<false, false><<<grid, 256, kGemmSmem, st>>>(Ab, d, U + r0 * d, d, U + (r0 + kw) * d, d, rest,
                                                               r0 + kw, (int)kw, vec16(Ab, d), 0);
     }
     e = cudaGetLastError();
@@ -764,6 +806,7 @@ cudaError_t launch_sketch_round(const float* theta, const double* U, const uint1
   round_init_kernel<<<(unsigned)(num_sms() * 8), 256, 0, st>>>(theta, n * d, W);
   cudaError_t e = cudaFuncSetAttribute(round_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        RB * RB * (int)sizeof(double));
+  if (e == cudaSuccess) e = gemm_smem_setup();
   if (e != cudaSuccess) return e;
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -775,7 +818,7 @@ cudaError_t launch_sketch_round(const float* theta, const double* U, const uint1
     const int64_t rest = d - j0 - kb;
     if (rest > 0) {
       dim3 grid((unsigned)cdiv(rest, GT), (unsigned)cdiv(n, GT));
-      gemm_sub_f64_kernel<false, false><<<grid, 256, 0, st>>>(E, RB, U + j0 * d + j0 + RB, d, W + j0 + RB, d, n, rest,
+      gemm_sub_f64_kernel<false, false><<<grid, 256, kGemmSmem, st>>>(E, RB, U + j0 * d + j0 + RB, d, W + j0 + RB, d, n, rest,
                                                               RB, vec16(E, RB), 0);
     }
     e = cudaGetLastError();
