@@ -625,7 +625,8 @@ def run_sketch(args, w, rank, device):
     used = [li for _, m in sketch_inputs() for li in m]
     weights = sum(shapes[li][0] * shapes[li][1] for li in used)
     # algorithmic work per stage and step
-    work = {"gram": sum(2.0 * s_tok * shapes[m[0]][1] ** 2 for _, m in sketch_inputs()),
+    # (the Gram matrix is symmetric: its upper triangle, s * d * (d + 1) flops)
+    work = {"gram": sum(float(s_tok) * shapes[m[0]][1] * (shapes[m[0]][1] + 1) for _, m in sketch_inputs()),
             "factor": sum(2.0 / 3.0 * shapes[m[0]][1] ** 3 for _, m in sketch_inputs()),
             "round": sum(float(shapes[li][0]) * shapes[li][1] ** 2 for li in used)}
     res = dict(ms=ms, per_stage=per_stage, work=work, weights=weights, clocks=clocks)

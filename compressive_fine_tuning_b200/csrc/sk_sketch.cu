@@ -55,11 +55,15 @@ constexpr uint32_t IDESC = tc::idesc_bf16(M, N, 1, 1);
 constexpr int TMEM_COLS = 256;
 }  // namespace gr
 
-// H[i0:i0+128][j0:j0+256] (+)= sum_t X[t][i] X[t][j]
+// H[i0:i0+128][j0:j0+256] (+)= sum_t X[t][i] X[t][j].  H is symmetric, so
+// only tiles that touch the upper triangle (j >= i) run; their epilogue
+// writes each upper element H[i][j] and its mirror H[j][i] (for a fixed
+// column the warp's 32 rows make one coalesced 128-byte store).
 __global__ void __launch_bounds__(gr::THREADS, 1)
 gram_tc_kernel(const __grid_constant__ CUtensorMap tm_x, int64_t s, int64_t d, float* __restrict__ H, int accumulate,
                unsigned int* check) {
   using namespace gr;
+  if ((int64_t)blockIdx.x * N + N - 1 < (int64_t)blockIdx.y * M) return;   // entirely below the diagonal
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
@@ -143,23 +147,20 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_x, int64_t s, int64_t d, f
         for (int e = 0; e < 32; ++e) v[e] = 0u;
       }
       if (i < d && (have || nsteps == 0)) {
-        float* dst = H + i * d + jc;
         const int cnt = (int)(d - jc < 32 ? d - jc : 32);
-        if (cnt == 32 && (d % 4) == 0) {
+        // the upper part of the row (j >= i) and the mirrors of j > i
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            float4 o = make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]), __uint_as_float(v[e + 2]),
-                                   __uint_as_float(v[e + 3]));
-            if (accumulate) {
-              const float4 old = *reinterpret_cast<const float4*>(dst + e);
-              o.x += old.x; o.y += old.y; o.z += old.z; o.w += old.w;
+        for (int e = 0; e < 32; ++e) {
+          const int64_t j = jc + e;
+          if (e < cnt && j >= i) {
+            const float val = __uint_as_float(v[e]);
+            float* up = H + i * d + j;
+            *up = (accumulate ? *up : 0.f) + val;
+            if (j > i) {
+              float* lo = H + j * d + i;
+              *lo = (accumulate ? *lo : 0.f) + val;
             }
-            *reinterpret_cast<float4*>(dst + e) = o;
           }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (e < cnt) dst[e] = (accumulate ? dst[e] : 0.f) + __uint_as_float(v[e]);
         }
       }
     }
