@@ -216,31 +216,34 @@ __global__ void reverse_damp_kernel(const float* __restrict__ H, int64_t d, cons
 // Unblocked Cholesky of the diagonal block A[k0:k0+kb][k0:k0+kb] (lower) in
 // shared memory; a pivot that is not positive flags the check word (the
 // factor then holds NaNs)
-__global__ void __launch_bounds__(256) potrf_diag_kernel(double* __restrict__ A, int64_t d, int64_t k0, int kb,
+__global__ void __launch_bounds__(1024) potrf_diag_kernel(double* __restrict__ A, int64_t d, int64_t k0, int kb,
                                                          unsigned int* check) {
   __shared__ double a[NB][NB + 1];
+  __shared__ double diag[NB];
   for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
     const int r = e / NB, c = e % NB;
     a[r][c] = (r < kb && c <= r) ? A[(k0 + r) * d + k0 + c] : 0.0;
   }
   __syncthreads();
   for (int c = 0; c < kb; ++c) {
+    // every thread derives the pivot from a[c][c], which nothing writes during
+    // this step (the factor's diagonal goes to diag[] and back at the end);
+    // the column below is scaled by the pivot's reciprocal
+    const double p = a[c][c];
+    const double piv = sqrt(p), rp = 1.0 / piv;
     if (threadIdx.x == 0) {
-      const double p = a[c][c];
       if (!(p > 0.0)) atomicOr(check, SK_CHECK_NOT_SPD);
-      a[c][c] = sqrt(p);
+      diag[c] = piv;
     }
+    for (int r = c + 1 + (int)threadIdx.x; r < kb; r += blockDim.x) a[r][c] *= rp;
     __syncthreads();
-    const double piv = a[c][c];
-    for (int r = c + 1 + (int)threadIdx.x; r < kb; r += blockDim.x) a[r][c] /= piv;
-    __syncthreads();
-    for (int r = c + 1 + (int)(threadIdx.x >> 4); r < kb; r += 16)
-      for (int q = c + 1 + (int)(threadIdx.x & 15); q <= r; q += 16) a[r][q] -= a[r][c] * a[q][c];
+    for (int r = c + 1 + (int)(threadIdx.x >> 5); r < kb; r += 32)
+      for (int q = c + 1 + (int)(threadIdx.x & 31); q <= r; q += 32) a[r][q] -= a[r][c] * a[q][c];
     __syncthreads();
   }
   for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
     const int r = e / NB, c = e % NB;
-    if (r < kb && c <= r) A[(k0 + r) * d + k0 + c] = a[r][c];
+    if (r < kb && c <= r) A[(k0 + r) * d + k0 + c] = r == c ? diag[r] : a[r][c];
   }
 }
 
@@ -248,10 +251,12 @@ __global__ void __launch_bounds__(256) potrf_diag_kernel(double* __restrict__ A,
 // x with x L_kk^T = a (forward substitution), one thread per row
 __global__ void __launch_bounds__(64) trsm_panel_kernel(double* __restrict__ A, int64_t d, int64_t k0) {
   __shared__ double l[NB][NB + 1];
+  __shared__ double rdiag[NB];
   for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
     const int r = e / NB, c = e % NB;
     l[r][c] = c <= r ? A[(k0 + r) * d + k0 + c] : 0.0;
   }
+  for (int c = threadIdx.x; c < NB; c += blockDim.x) rdiag[c] = 1.0 / A[(k0 + c) * d + k0 + c];
   __syncthreads();
   const int64_t r = k0 + NB + (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (r >= d) return;
@@ -259,13 +264,14 @@ __global__ void __launch_bounds__(64) trsm_panel_kernel(double* __restrict__ A, 
   double x[NB];
 #pragma unroll
   for (int c = 0; c < NB; ++c) x[c] = row[c];
-  // the dot products run as four interleaved partial sums (shorter dependency chains)
+  // right-looking: once x_c is final it is removed from every later entry,
+  // so each step's updates are independent and only one multiply per column
+  // sits on the critical path
 #pragma unroll
   for (int c = 0; c < NB; ++c) {
-    double p[4] = {0.0, 0.0, 0.0, 0.0};
+    x[c] *= rdiag[c];
 #pragma unroll
-    for (int q = 0; q < c; ++q) p[q & 3] = fma(x[q], l[c][q], p[q & 3]);
-    x[c] = (x[c] - ((p[0] + p[1]) + (p[2] + p[3]))) / l[c][c];
+    for (int q = c + 1; q < NB; ++q) x[q] = fma(-x[c], l[q][c], x[q]);
   }
 #pragma unroll
   for (int c = 0; c < NB; ++c) row[c] = x[c];
@@ -410,10 +416,13 @@ __global__ void __launch_bounds__(64) trtri_rows_kernel(const double* __restrict
                                                         int64_t d, int64_t r0, int kb) {
   if (FULL) kb = NB;
   __shared__ double l[NB][NB + 1];
+  __shared__ double rdiag[NB];
   for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
     const int r = e / NB, c = e % NB;
     l[r][c] = (r < kb && c <= r) ? L[(r0 + r) * d + r0 + c] : (r == c ? 1.0 : 0.0);
   }
+  __syncthreads();
+  for (int r = threadIdx.x; r < NB; r += blockDim.x) rdiag[r] = 1.0 / l[r][r];
   __syncthreads();
   const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (c >= r0 + kb) return;
@@ -424,12 +433,12 @@ __global__ void __launch_bounds__(64) trtri_rows_kernel(const double* __restrict
     x[r] = r < kb ? *src : 0.0;
     src += d;
   }
+  // right-looking, as in the panel solve
 #pragma unroll
   for (int r = 0; r < NB; ++r) {
-    double p[4] = {0.0, 0.0, 0.0, 0.0};
+    x[r] *= rdiag[r];
 #pragma unroll
-    for (int q = 0; q < r; ++q) p[q & 3] = fma(l[r][q], x[q], p[q & 3]);
-    x[r] = (x[r] - ((p[0] + p[1]) + (p[2] + p[3]))) / l[r][r];
+    for (int q = r + 1; q < NB; ++q) x[q] = fma(-l[q][r], x[r], x[q]);
   }
   double* dst = Mx + r0 * d + c;
 #pragma unroll
@@ -585,7 +594,7 @@ lloyd_kernel(const float* __restrict__ theta, const double* __restrict__ hinv, i
 // 4. column-by-column mapping with error compensation
 // ============================================================================
 
-constexpr int kRoundWarps = 16;   // rows per CTA, one warp each
+constexpr int kRoundWarps = 32;   // rows per CTA, one warp each
 constexpr int RB = 128;           // columns per mapping block (the rank of its lazy update)
 constexpr int RQ = RB / 32;       // columns per lane
 
@@ -721,7 +730,7 @@ cudaError_t launch_inverse_factor(const float* H, int64_t d, double damp, double
       const int64_t kk = k0 + h * NB;
       if (kk >= d) break;
       const int kb = (int)(d - kk < NB ? d - kk : NB);
-      potrf_diag_kernel<<<1, 256, 0, st>>>(A, d, kk, kb, check);
+      potrf_diag_kernel<<<1, 1024, 0, st>>>(A, d, kk, kb, check);
       const int64_t rest = d - kk - kb;
       if (rest > 0) trsm_panel_kernel<<<(unsigned)cdiv(rest, 64), 64, 0, st>>>(A, d, kk);
       if (h == 0 && rest > 0) {
