@@ -526,6 +526,29 @@ def run_ours(args, w, rank, world, device):
 # the sketching stage (dense weights + calibration activations -> sketch)
 # ---------------------------------------------------------------------------
 
+def sketch_factor_launches(d, nb=64):
+    """Kernel launches of one inverse factor of a d x d Gram matrix (the
+    launch loops of the library, counted)."""
+    n = 2                                              # damping, reversal
+    for k0 in range(0, d, 2 * nb):                     # Cholesky super-blocks
+        for h in range(2):
+            kk = k0 + h * nb
+            if kk >= d:
+                break
+            rest = d - kk - min(nb, d - kk)
+            n += 1 + (1 if rest > 0 else 0) + (1 if h == 0 and rest > 0 else 0)
+        n += 1 if d - k0 - min(d - k0, 2 * nb) > 0 else 0
+    n += 1                                             # identity
+    for r0 in range(0, d, 2 * nb):                     # inverse super-blocks
+        for h in range(2):
+            rr = r0 + h * nb
+            if rr >= d:
+                break
+            n += 1 + (1 if h == 0 and d - rr - min(nb, d - rr) > 0 else 0)
+        n += 1 if d - r0 - min(d - r0, 2 * nb) > 0 else 0
+    return n + 2                                       # reversal, column norms
+
+
 def sketch_cpu_baseline(budget_rows=32, tokens=4096, seed=0):
     """The oracle's sketching stage on a bounded sample: the q_proj input with
     `tokens` calibration tokens (Gram matrix and inverse factor of the full
@@ -718,16 +741,14 @@ def main_sketch(args, w, world, rank, local):
     roof["stages_ms"] = st
     roof["stage_rates_tflops"] = rates
     roof["fp64_peak_tflops"] = fp64_peak
-    n_launch = 0
     from compressive_fine_tuning_b200 import synth
     shapes = synth.LLAMA2_7B
+    n_launch = 0
     for _, members in sketch_inputs():
-        d = shapes[members[0]][1]
-        nb = (d + 63) // 64
-        n_launch += 1 + 2 + 3 * nb - 2 + 1 + 2 * nb - 1 + 2   # Gram; damping; Cholesky; identity; inverse; reverse, norms
+        n_launch += 1 + sketch_factor_launches(shapes[members[0]][1])          # Gram, inverse factor
         for li in members:
-            nbl = (shapes[li][1] + 63) // 64
-            n_launch += 1 + 1 + 2 * nbl - 1 + 1                 # Lloyd; copy; mapping blocks and GEMMs; pack
+            nr = (shapes[li][1] + 127) // 128
+            n_launch += 1 + 1 + nr + (nr - 1) + 1                              # Lloyd; copy; blocks, GEMMs; pack
     line = {"metric": SKETCH_METRIC, "value": res["weights"] * world / (step_ms / 1e3), "unit": unit,
             "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
