@@ -17,6 +17,14 @@ Two ways the layer shards, and the one exchange that either needs:
   task's LUT rows of its slice and computes its slice of Y with no exchange.
   Only a consumer that wants the whole Y gathers the slices.
 
+* The sketching stage shards its calibration tokens and then its rows.  The
+  Gram matrix is a sum over tokens, so each rank computes it over its own
+  calibration shard and one all-reduce (d * d * 4 bytes) gives everyone the
+  whole matrix; every rank then factors it (the same launches on the same
+  data) and runs Lloyd and the mapping for its own slice of weight rows,
+  which need nothing from the other rows.  Only a consumer that wants the
+  whole index map or all the LUTs gathers the row blocks.
+
 Everything here is host logic over ``torch.distributed``; the arithmetic runs
 in the library's kernels.  The functions accept CPU tensors too (``gloo``), so
 the exchange logic can be exercised without a GPU.
@@ -113,3 +121,30 @@ def gather_rows(y_local: torch.Tensor, n: int, group: Optional[dist.ProcessGroup
     parts = [torch.empty_like(buf) for _ in range(world)]
     dist.all_gather(parts, buf.contiguous(), group=group)
     return torch.cat([p[:, : s.stop - s.start] for p, s in zip(parts, widths)], dim=1)
+
+
+def reduce_gram(H: torch.Tensor, group: Optional[dist.ProcessGroup] = None) -> torch.Tensor:
+    """Sum, in place, the Gram matrices that the ranks computed over their
+    shards of the calibration tokens (sk.gram of the local rows of X).  The
+    summation order of the all-reduce is the library's, so the sum can differ
+    from a single-device Gram matrix in the last bits."""
+    if dist.get_world_size(group) > 1:
+        dist.all_reduce(H, op=dist.ReduceOp.SUM, group=group)
+    return H
+
+
+def gather_row_blocks(x_local: torch.Tensor, n: int, group: Optional[dist.ProcessGroup] = None,
+                      align: int = 8) -> torch.Tensor:
+    """Concatenate every rank's block of rows [rows of its shard][...] (the
+    rows of `row_shard`) into [n][...], e.g. the index map or the LUTs that
+    the ranks sketched for their own rows."""
+    world = dist.get_world_size(group)
+    if world == 1:
+        return x_local
+    shards = [row_shard(n, r, world, align) for r in range(world)]
+    rows_max = max(sh.stop - sh.start for sh in shards)
+    buf = x_local.new_zeros((rows_max,) + tuple(x_local.shape[1:]))
+    buf[: x_local.shape[0]] = x_local
+    parts = [torch.empty_like(buf) for _ in range(world)]
+    dist.all_gather(parts, buf.contiguous(), group=group)
+    return torch.cat([p[: sh.stop - sh.start] for p, sh in zip(parts, shards)], dim=0)

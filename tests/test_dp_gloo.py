@@ -3,7 +3,9 @@
 The exchange logic of compressive_fine_tuning_b200.dp is exercised with the
 oracle standing in for each rank's kernels: the sum of per-rank LUT gradients
 over a token-sharded batch must equal the gradient of the whole batch, and the
-row-sharded forward, gathered, must equal the unsharded forward.
+row-sharded forward, gathered, must equal the unsharded forward, and the
+sketching stage sharded over calibration tokens and then rows must give the
+same index map and LUTs as one process.
 """
 import os
 import socket
@@ -62,6 +64,34 @@ def _fwd_worker(rank, world, port):
         assert np.array_equal(y.numpy(), full)
     finally:
         dist.destroy_process_group()
+
+
+def _sketch_worker(rank, world, port):
+    """Calibration tokens sharded for the Gram matrix (one all-reduce), rows
+    sharded for Lloyd and the mapping, row blocks gathered: the same index map
+    and LUTs as the whole stage on one process."""
+    _init(rank, world, port)
+    try:
+        n, d, gpr, bits = 24, 64, 2, 2
+        c = synth.sketch_case(21, n, d, 300)
+        idx_ref, lut_ref = oracle.sketch_layer(c.theta, c.x, bits, gpr)
+        toks = dp.token_shard(c.s, rank, world)
+        h = dp.reduce_gram(torch.from_numpy(oracle.gram(c.x[toks])))
+        np.testing.assert_allclose(h.numpy(), oracle.gram(c.x), rtol=1e-12, atol=1e-9)
+        u, hd = oracle.inverse_factor(oracle.damped(h.numpy(), 0.01))
+        rows = dp.row_shard(n, rank, world)
+        lut_loc = oracle.lloyd_luts(c.theta[rows], hd, bits, gpr, 100)
+        idx_loc = oracle.sketch_round(c.theta[rows], u, lut_loc)
+        lut = dp.gather_row_blocks(torch.from_numpy(lut_loc), n).numpy()
+        idx = dp.gather_row_blocks(torch.from_numpy(idx_loc), n).numpy()
+        assert np.array_equal(lut.view(np.uint16), lut_ref.view(np.uint16))
+        assert np.array_equal(idx, idx_ref)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sketching_stage_shards_tokens_then_rows():
+    mp.spawn(_sketch_worker, args=(2, _free_port()), nprocs=2, join=True)
 
 
 @pytest.mark.parametrize("ntask,average", [(1, False), (3, False), (1, True)])
