@@ -37,6 +37,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -199,7 +200,10 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+        # the samples go to a scratch file next to the run (SK_CLOCKS_DIR, else
+        # the system temporary directory)
+        base = os.environ.get("SK_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(base, f"clocks_gpu{gpu_index}_{os.getpid()}.csv")
 
     def start(self):
         try:
