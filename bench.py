@@ -516,8 +516,7 @@ def run_ours(args, w, rank, world, device):
         h2d = sum(t.numel() * t.element_size() for ent in in_views.values() for (_, t) in ent.values())
         d2h = sum(t.numel() * t.element_size() for (_, t) in out_views.values())
         # transfers are issued in pieces of at most 64 MiB (one piece for a
-        # decode step): single copies of several hundred MB ran at about 36 GB/s
-        # on this bus against about 56 GB/s in pieces of this size
+        # decode step)
         piece = 64 << 20
 
         def copy_in_pieces(dst, src):
