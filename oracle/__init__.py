@@ -25,7 +25,7 @@ from .sketch_oracle import (  # noqa: F401
     row_stride_bytes, packed_bytes, pack, unpack, dequant, sketch_matrix,
     dequant_via_sketch_matrix, forward, backward_input, backward_lut,
     eq6_forward, eq6_backward_lut, bin_counts, trainable_params, lora_params,
-    compression_factor, averaged_gradient, adamw_step, sgd_step,
+    compression_factor, averaged_gradient, adamw_step, sgd_step, sketched_model_bytes,
 )
 from .sketching_oracle import (  # noqa: F401
     gram, damped, inverse_factor, lloyd_init, lloyd_assign, lloyd_update, lloyd,

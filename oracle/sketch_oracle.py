@@ -322,3 +322,12 @@ def lora_params(shapes, layers: int, r: int) -> int:
 def compression_factor(c: int, g: int, k: int) -> float:
     """A row of c values sketched into g groups of k entries ("Sketch to Adapt", reply W2)."""
     return c / (g * k)
+
+
+def sketched_model_bytes(shapes, layers: int, bits: int, gpr: int, dense_params: int = 0) -> int:
+    """Bytes of a sketched model: per matrix the packed indices (n * d * bits /
+    8) and one fp16 LUT set (n * gpr * 2**bits * 2), summed over the layers,
+    plus `dense_params` fp16 parameters kept unsketched (embeddings, head)."""
+    k = 1 << bits
+    per_layer = sum(n * d * bits // 8 + n * gpr * k * 2 for n, d in shapes)
+    return layers * per_layer + 2 * dense_params

@@ -325,6 +325,10 @@ def test_page_counts():
     v, _ = counts["min_compression_factor_7b"]
     factors = [oracle.compression_factor(c, g, k) for c in (4096, 11008) for g in (1, 2, 4, 8) for k in (4, 8, 16)]
     assert min(factors) == v
+    v, tol = counts["llama3_70b_4bit_gpr4_bytes"]
+    got = oracle.sketched_model_bytes(synth.LLAMA3_70B, 80, 4, 4, dense_params=2 * 128256 * 8192)
+    idx_bytes = 80 * sum(n * d for n, d in synth.LLAMA3_70B) // 2
+    assert idx_bytes == 34_225_520_640 and abs(got - v) <= tol
 
 
 # ---------------------------------------------------------------------------
