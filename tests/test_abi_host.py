@@ -222,3 +222,41 @@ def test_sketch_without_device_fails_loudly():
     assert L.sk_lloyd(A, B, 4, 1, 8, 64, 10, C, None, None) in (SK_ERR_CUDA, SK_ERR_UNSUPPORTED)
     assert L.sk_sketch_round(A, B, C, 4, 1, 8, 64, D, E, L.sk_sketch_round_workspace_bytes(8, 64), None) in (
         SK_ERR_CUDA, SK_ERR_UNSUPPORTED)
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include "sk.h"
+
+/* a plain C caller: header compiles as C, symbols link without C++ mangling,
+   and host-side validation answers before any device work */
+int main(void) {
+  if (sk_abi_version() != SK_ABI_VERSION) return 1;
+  if (sk_packed_row_bytes(4096, 4) != 2048) return 2;
+  if (sk_packed_bytes(7, 96, 3) != 7 * 48) return 3;
+  if (sk_linear_fwd(NULL, NULL, 4, 1, 256, 512, NULL, 4, NULL, 1, NULL, NULL, 0, NULL) != SK_ERR_INVALID_ARG) return 4;
+  if (sk_gram(NULL, 16, 60, NULL, 0, NULL) != SK_ERR_INVALID_ARG) return 5;
+  if (sk_last_error()[0] == 0) return 6;
+  printf("%s\n", sk_status_string(SK_ERR_INVALID_ARG));
+  return 0;
+}
+"""
+
+
+def test_c_caller_links_and_validates(tmp_path):
+    """The header is valid C and the library links into a C program."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "caller.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(sk._LIB_PATH)
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                        "-L", libdir, "-lsk", f"-Wl,-rpath,{libdir}"], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    assert r.stdout.strip() == "SK_ERR_INVALID_ARG"
