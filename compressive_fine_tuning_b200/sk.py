@@ -378,3 +378,32 @@ class SketchedLinearFunction(torch.autograd.Function):
 def sketched_linear(X: torch.Tensor, lut: torch.Tensor, packed: torch.Tensor, bits: int,
                     task: Optional[torch.Tensor] = None) -> torch.Tensor:
     return SketchedLinearFunction.apply(X, lut, packed, bits, task)
+
+
+class SketchedLinear(torch.nn.Module):
+    """A linear layer (no bias) whose weight is the sketch Theta_hat: a frozen
+    packed index map (buffer) and trainable fp16 LUTs [ntask, n, gpr, 2**bits]
+    (parameter).  forward(X, task) takes bf16 activations [..., d]; task holds
+    one LUT-set id per token (int32), or None for set 0."""
+
+    def __init__(self, packed: torch.Tensor, lut: torch.Tensor, bits: int, in_features: int):
+        super().__init__()
+        self.register_buffer("packed", packed)
+        self.lut = torch.nn.Parameter(lut)
+        self.bits = bits
+        self.in_features = in_features
+        self.out_features = lut.shape[1]
+
+    @classmethod
+    def from_dense(cls, weight: torch.Tensor, X_calib: torch.Tensor, bits: int, gpr: int, ntask: int = 1,
+                   damp: float = 0.01, max_iter: int = 100) -> "SketchedLinear":
+        """Sketch a dense weight [n, d] with calibration activations [s, d]
+        (bf16); every LUT set starts from the same learned centroids."""
+        packed, lut, _ = sketch_layer(weight.float().contiguous(), X_calib, bits, gpr, damp, max_iter)
+        return cls(packed, lut.unsqueeze(0).repeat(ntask, 1, 1, 1).contiguous(), bits, weight.shape[1])
+
+    def forward(self, X: torch.Tensor, task: Optional[torch.Tensor] = None) -> torch.Tensor:
+        lead = X.shape[:-1]
+        Y = sketched_linear(X.reshape(-1, self.in_features).to(torch.bfloat16).contiguous(), self.lut, self.packed,
+                            self.bits, task)
+        return Y.reshape(*lead, self.out_features)

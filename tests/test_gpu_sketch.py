@@ -293,3 +293,28 @@ def test_identity_is_sketched_exactly_on_the_device(bits):
     x = synth.make_calib(synth.rng_for(61000), 512, d)
     packed, lut, idx = _sk().sketch_layer(torch.eye(d, device="cuda"), _bf16(x), bits, 1)
     np.testing.assert_array_equal(oracle.dequant(idx.cpu().numpy(), lut.cpu().numpy()), np.eye(d))
+
+
+def test_sketched_linear_module_from_dense():
+    """SketchedLinear.from_dense runs the stage on the device; its forward and
+    LUT gradient match the oracle evaluated on the module's own index map and
+    LUTs, and two LUT sets route per token."""
+    from tests import gpu_cases as gc
+    sk = _sk()
+    n, d, gpr, bits, T = 128, 256, 2, 4, 96
+    c = synth.sketch_case(61100, n, d, 1024)
+    mod = sk.SketchedLinear.from_dense(torch.from_numpy(c.theta).cuda(), _bf16(c.x_bits), bits, gpr, ntask=2)
+    idx = sk.unpack(mod.packed, n, d, bits).cpu().numpy()
+    lut = mod.lut.detach().cpu().numpy()
+    rng = synth.rng_for(61101)
+    xb = synth.make_bf16(rng, (T, d), synth.X_STD)
+    task = synth.make_task(rng, T, 2)
+    X = _bf16(xb)
+    Y = mod(X, torch.from_numpy(task).cuda())
+    ref = oracle.forward(synth.bf16_bits_to_f64(xb), idx, lut, task)
+    absb = np.abs(synth.bf16_bits_to_f64(xb)) @ np.abs(oracle.dequant(idx, lut[0])).T
+    gc.check_rows(gc.bf16_to_f64(Y), ref, absb, "module forward")
+    Y.float().sum().backward()
+    dl_ref = oracle.backward_lut(synth.bf16_bits_to_f64(xb), np.ones((T, n)), idx, gpr, 1 << bits, task=task, ntask=2)
+    got = mod.lut.grad.float().cpu().numpy()
+    assert np.linalg.norm(got - dl_ref) <= 2e-3 * np.linalg.norm(dl_ref)
