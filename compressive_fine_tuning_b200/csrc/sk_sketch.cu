@@ -7,25 +7,28 @@
 // step followed by an update of the parameters not yet mapped).
 //
 //   1. H = X^T X: a tcgen05 GEMM over the calibration tokens, both operands
-//      MN-major straight from TMA, fp32 accumulators in TMEM;
+//      MN-major straight from TMA, fp32 accumulators in TMEM; only the tiles
+//      that touch the upper triangle run, and they also write the mirror;
 //   2. damping and the inverse factor U (H^-1 = U^T U, U upper), in float64:
 //      the index-reversed H is factored by a blocked Cholesky (diagonal
-//      block in one CTA, panel solve one thread per row, trailing update as a
-//      GEMM), the lower factor is inverted by blocked forward substitution,
-//      and reversing the indices of that inverse gives U; diag(H^-1) is the
-//      column sums of squares of U;
+//      block in one CTA, panel solve one thread per row, trailing updates as
+//      GEMMs of rank 64 inside and 128 across super-blocks of two blocks),
+//      the lower factor is inverted by blocked forward substitution in the
+//      same super-blocks, and reversing the indices of that inverse gives U;
+//      diag(H^-1) is the column sums of squares of U;
 //   3. weighted Lloyd per (row, group), one CTA each: the group's values are
 //      sorted once in shared memory, so a cluster is a contiguous range and
 //      an assignment is k - 1 binary searches against float32 midpoints;
 //      each warp sums one cluster in float64;
-//   4. the mapping in blocks of 64 columns: one warp per row walks the
+//   4. the mapping in blocks of 128 columns: one warp per row walks the
 //      block's columns in order (nearest fp16 centroid by float32 midpoints,
 //      then the compensation of the block's later columns), and a float64
 //      GEMM applies the block's compensation to every later column.
 //
-// Everything after the Gram matrix is float64, so the integer decisions
-// (clusters, centroids chosen) agree with a float64 evaluation except for
-// values within rounding distance of a midpoint.
+// After the Gram matrix all sums and carried values are float64 and every
+// integer decision (a cluster, a chosen centroid) compares a value with a
+// float32 midpoint, so the decisions agree with a float64 evaluation except
+// for values within rounding distance of a midpoint.
 #include <cfloat>
 #include <cmath>
 
@@ -178,7 +181,7 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_x, int64_t s, int64_t d, f
 // 2. float64 linear algebra: damping, blocked Cholesky, triangular inverse
 // ============================================================================
 
-constexpr int NB = 64;   // block size of the factorizations and of the mapping
+constexpr int NB = 64;   // block size of the factorizations (two of them form a super-block)
 
 // lambda = damp * mean(diag H), a zero diagonal entry counted as 1; one CTA,
 // fixed summation order
