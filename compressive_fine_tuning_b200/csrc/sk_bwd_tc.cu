@@ -598,8 +598,12 @@ cudaError_t launch_dlut_tc_routed(const Problem& p, const uint16_t* X, const uin
 // its memory up front and treats any new allocation as an error, or code that
 // must not call cudaMalloc because it synchronises the device.  For them the
 // partial bins live in one file-scope device array instead of a caller
-// workspace.  The array is reserved on every GPU that loads this library and is
-// held until the process exits.
+// workspace.  The array belongs to this file's device module, so it is
+// reserved on a device as soon as that module is loaded there -- on the first
+// use of any kernel of this file (the tensor-core input and LUT gradients) or
+// of the allocation-free call, or when the context is created if modules load
+// eagerly -- and it is held until the process exits, whether or not the
+// allocation-free call is ever made.
 #include <mutex>
 
 namespace sk {
@@ -609,8 +613,21 @@ constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kNoAllocMaxDevices = 64;
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
 std::mutex g_noalloc_mutex;
+std::once_flag g_ctx_once;
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+// per device: the context the address was looked up in, and the address
+CUcontext g_noalloc_ctx[kNoAllocMaxDevices] = {};
 void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+void load_ctx_get_current() {
+  cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+  void* fn = nullptr;
+  if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+}
 
 }  // namespace
 
@@ -618,18 +635,25 @@ size_t dlut_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
 
 // Device address of the scratch array on the current device.  In host code the
 // array's name only stands for the host-side shadow symbol, so the device
-// address is looked up once per device (with that device current) and cached.
+// address is looked up with the device current.  The lookup is cached per
+// device together with the context it was made in: if that context has been
+// torn down and replaced (a device reset), the module is loaded again at a
+// possibly different address and the lookup is repeated.
 cudaError_t dlut_noalloc_scratch(void** ptr) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
+  std::call_once(g_ctx_once, load_ctx_get_current);
+  CUcontext ctx = nullptr;
+  if (g_ctx_get_current == nullptr || g_ctx_get_current(&ctx) != CUDA_SUCCESS) ctx = nullptr;
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  if (g_noalloc_ptr[dev] == nullptr || ctx == nullptr || ctx != g_noalloc_ctx[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
     g_noalloc_ptr[dev] = p;
+    g_noalloc_ctx[dev] = ctx;
   }
   *ptr = g_noalloc_ptr[dev];
   return cudaSuccess;

@@ -190,15 +190,21 @@ sk_status sk_linear_bwd_lut(const void* packed, int bits, int gpr, int64_t n, in
  * counterpart: this is a deployment convenience of this library.
  *
  * It allocates nothing: where sk_linear_bwd_lut would take a caller workspace,
- * this call uses one fixed array of SK_NOALLOC_SCRATCH_BYTES in device memory,
- * reserved on every GPU that loads the library until the process exits.  The
- * caller still passes the inputs and dlut.  Arguments, layouts, results and
+ * this call uses one fixed array of SK_NOALLOC_SCRATCH_BYTES (32 MiB) in
+ * device memory.  The array is part of the library's backward-kernel module:
+ * a process holds those 32 MiB on every device where that module is loaded
+ * (the first tensor-core input or LUT gradient, or the first call of this
+ * function, on that device; every device the library initialises when CUDA
+ * loads modules eagerly), until it exits, whether or not it ever calls this
+ * function.  The caller still passes the inputs and dlut.  Arguments, layouts, results and
  * errors are those of sk_linear_bwd_lut; in addition a layer whose scratch
  * need (sk_workspace_bytes(SK_OP_BWD_LUT, ...)) exceeds the array is rejected
  * with SK_ERR_INVALID_ARG before anything is launched.
  *
  * The first call on a device looks up the array's device address with that
- * device current; make that first call before any stream capture.  Every call
+ * device current; make that first call before any stream capture.  The
+ * address is cached per device and context: after a device reset the next
+ * call looks it up again (again outside any stream capture).  Every call
  * shares the one array and it keeps the last call's contents (each call
  * overwrites every entry it reads, so nothing has to start at zero): calls that
  * overlap on the GPU (different streams, concurrently replayed graphs) race and

@@ -260,3 +260,36 @@ def test_c_caller_links_and_validates(tmp_path):
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
     assert r.stdout.strip() == "SK_ERR_INVALID_ARG"
+
+
+NOALLOC_REJECT = r"""
+import ctypes, sys
+sys.path.insert(0, sys.argv[1])
+from compressive_fine_tuning_b200 import sk
+# the 70B gate projection at 4 bits and 4 groups per row needs more partial-bin
+# scratch than the allocation-free call holds, whatever the batch
+n, d, bits, gpr, T = 28672, 8192, 4, 4, 64
+need = sk.workspace_bytes(sk.SK_OP_BWD_LUT, n, d, bits, gpr, T, 1)
+assert need > (32 << 20), need
+p = [ctypes.c_void_p(a) for a in (0x10000000, 0x20000000, 0x40000000, 0x80000000)]
+st = sk.lib.sk_linear_bwd_lut_noalloc(p[0], bits, gpr, n, d, p[1], p[2], T, None, 1, p[3], 0, None)
+print(st, sk.lib.sk_last_error().decode())
+"""
+
+
+def test_noalloc_rejects_layers_beyond_its_scratch():
+    """The allocation-free LUT gradient refuses, on the host, a layer whose
+    partial bins exceed its fixed array.  The call runs in a child process that
+    sees no CUDA device and keeps the library's own kernel choice, so even a
+    broken size check could only fail on the missing device: nothing can be
+    launched against the made-up addresses."""
+    import subprocess
+    import sys
+    env = {k: v for k, v in os.environ.items() if k != "SK_BWD_PATH"}
+    env["CUDA_VISIBLE_DEVICES"] = ""
+    r = subprocess.run([sys.executable, "-c", NOALLOC_REJECT, ROOT], capture_output=True, text=True, env=env,
+                       timeout=300)
+    assert r.returncode == 0, r.stderr
+    st, msg = r.stdout.strip().split(" ", 1)
+    assert int(st) == SK_ERR_INVALID_ARG
+    assert "scratch" in msg

@@ -2,11 +2,14 @@
 
 It exists for callers that cannot allocate device memory when they need the
 gradient (for instance a plugin inside another framework's executor that owns
-every device allocation).  It must give the same result as the workspace-taking
-sk_linear_bwd_lut, within the LUT-gradient tolerance of the other parity
-tests, on consecutive calls that share its one scratch array.  This file is
-collected last so that a run stopping at the first failure has already run
-every other test; it also passes on its own in a fresh process.
+every device allocation, or a loop that has reserved its whole memory budget up
+front).  It must give the same result as the workspace-taking
+sk_linear_bwd_lut, and the oracle's, within the LUT-gradient tolerance of the
+other parity tests, on consecutive calls that share its one scratch array.
+This file is collected last so that a run stopping at the first failure has
+already run every other test; it also passes on its own in a fresh process.
+(The host-side rejection of layers too large for the array is tested without a
+device in tests/test_abi_host.py.)
 """
 import ctypes
 
@@ -18,6 +21,14 @@ torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
 
+@pytest.fixture(autouse=True)
+def _default_paths(monkeypatch):
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    # the kernel choice must be the library's own
+    monkeypatch.delenv("SK_BWD_PATH", raising=False)
+
+
 def _noalloc(sk, packed, bits, gpr, n, d, X, dY, T, out, accumulate=0, task=None, ntask=1):
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     return sk.lib.sk_linear_bwd_lut_noalloc(sk._ptr(packed), bits, gpr, n, d, sk._ptr(X), sk._ptr(dY), T,
@@ -25,8 +36,7 @@ def _noalloc(sk, packed, bits, gpr, n, d, X, dY, T, out, accumulate=0, task=None
 
 
 def test_noalloc_matches_workspace_call_on_consecutive_calls():
-    if not torch.cuda.is_available():
-        pytest.skip("no CUDA device")
+    import oracle
     from compressive_fine_tuning_b200 import sk, synth
     from tests import gpu_cases as gc
 
@@ -42,6 +52,8 @@ def test_noalloc_matches_workspace_call_on_consecutive_calls():
         assert _noalloc(sk, packed, bits, gpr, n, d, X, dY, T, got) == 0, sk.lib.sk_last_error()
         torch.cuda.synchronize()
         gc.check_dlut(got.cpu().numpy(), ref.cpu().numpy().astype(np.float64), "allocation-free dlut")
+        gc.check_dlut(got.cpu().numpy()[0], oracle.backward_lut(c.x, c.dy, c.idx, gpr, 1 << bits),
+                      "allocation-free dlut vs oracle")
         again = torch.full_like(ref, float("nan"))
         assert _noalloc(sk, packed, bits, gpr, n, d, X, dY, T, again) == 0
         torch.cuda.synchronize()
@@ -49,13 +61,37 @@ def test_noalloc_matches_workspace_call_on_consecutive_calls():
     assert sk.device_check() == 0
 
 
-def test_noalloc_rejects_layers_beyond_its_scratch():
-    from compressive_fine_tuning_b200 import sk
-    # a 70B-sized gate projection needs more partial-bin scratch than the fixed array
-    n, d, bits, gpr, T = 28672, 8192, 4, 4, 4096
-    need = sk.workspace_bytes(sk.SK_OP_BWD_LUT, n, d, bits, gpr, T, 1)
-    assert need > (32 << 20)
-    fake = [ctypes.c_void_p(a) for a in (0x10000000, 0x20000000, 0x40000000, 0x80000000)]
-    st = sk.lib.sk_linear_bwd_lut_noalloc(fake[0], bits, gpr, n, d, fake[1], fake[2], T, None, 1, fake[3], 0, None)
-    assert st == 1  # SK_ERR_INVALID_ARG, nothing launched
-    assert b"scratch" in sk.lib.sk_last_error()
+@pytest.mark.parametrize("kind", ["accumulate", "multitask", "few_tokens", "empty"])
+def test_noalloc_other_paths_match_oracle(kind):
+    """accumulate = 1 onto a non-zero gradient (tensor-core path), eight LUT
+    sets with task ids, a batch below the tensor-core threshold, and an empty
+    batch; each compared with the oracle, twice in a row."""
+    import oracle
+    from compressive_fine_tuning_b200 import sk, synth
+    from tests import gpu_cases as gc
+
+    n, d, bits, gpr = 512, 2048, 4, 4
+    T = {"accumulate": 256, "multitask": 200, "few_tokens": 32, "empty": 0}[kind]
+    ntask = 8 if kind == "multitask" else 1
+    c = synth.layer_case(21 + T, n=n, d=d, bits=bits, gpr=gpr, T=max(T, 1), ntask=ntask)
+    packed, lut, X, dY, task = gc.dev_case(c)
+    X, dY = X[:T], dY[:T]
+    if task is not None:
+        task = task[:T].contiguous()
+    ref = oracle.backward_lut(c.x[:T], c.dy[:T], c.idx, gpr, 1 << bits,
+                              task=None if c.task is None else c.task[:T], ntask=ntask)
+    ref = ref.reshape(ntask, n, gpr, 1 << bits)
+    start = np.full(ref.shape, 0.125) if kind in ("accumulate", "empty") else np.zeros(ref.shape)
+    acc = 1 if kind in ("accumulate", "empty") else 0
+    for _ in range(2):
+        out = torch.from_numpy(start.astype(np.float32)).cuda() if acc else torch.full(ref.shape, float("nan"),
+                                                                                      device="cuda")
+        st = _noalloc(sk, packed, bits, gpr, n, d, X, dY, T, out, accumulate=acc, task=task, ntask=ntask)
+        assert st == 0, sk.lib.sk_last_error()
+        torch.cuda.synchronize()
+        want = ref + (start if acc else 0.0)
+        if T == 0:
+            assert np.array_equal(out.cpu().numpy(), want.astype(np.float32))
+        else:
+            gc.check_dlut(out.cpu().numpy(), want, f"allocation-free dlut ({kind})")
+    assert sk.device_check() == 0
