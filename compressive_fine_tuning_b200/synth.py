@@ -41,9 +41,15 @@ def rng_for(seed: int) -> np.random.Generator:
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     """Round float32 values to bf16 (round-to-nearest-even); return raw uint16 bits."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    rounding_bias = ((u >> 16) & 1) + 0x7FFF
-    r = ((u + rounding_bias) >> 16).astype(np.uint16)
+    u = x.view(np.uint32)
+    # u + 0x7FFF + (bit 16 of u), in uint32: finite inputs stay below 2^32
+    # (the largest finite pattern is 0xFF7FFFFF)
+    t = u >> np.uint32(16)
+    t &= np.uint32(1)
+    t += np.uint32(0x7FFF)
+    t += u
+    t >>= np.uint32(16)
+    r = t.astype(np.uint16)
     nan = np.isnan(x)
     if nan.any():
         r[nan] = 0x7FC0
