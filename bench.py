@@ -75,6 +75,10 @@ WORKLOADS["sketch7b"] = dict(shapes="LLAMA2_7B", bits=4, gpr=8, batches=(128 * 2
 # 1965 MHz boost clock over 148 SMs); the fp64 stages report against this
 FP64_LANES_PER_SM = 64
 
+# the fine-tune workload measured beside the default decode workload: the
+# metric names both the LUT-GEMV bandwidth and the fwd+bwd throughput
+TRAIN_WORKLOAD = "finetune7b"
+
 L2_BYTES = 126 * 1024 * 1024
 # Integer-ALU cost of one 4-bit lookup (byte-permute network) and the integer
 # pipe's issue rate per SM on B200, measured with a throughput probe.
@@ -94,6 +98,8 @@ def parse():
                     help="comma-separated layer indices to run (a subset for profiling); default all")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-train", action="store_true",
+                    help="with the default decode workload, skip the fine-tune block (the metric's fwd+bwd half)")
     ap.add_argument("--launch-events", choices=("groups", "on", "off"), default="groups",
                     help="timing events captured between launches: 'groups' only where the kernel "
                          "changes (each event costs a few microseconds), 'on' between every launch")
@@ -293,6 +299,13 @@ def cpu_baseline(w, budget_s=15.0, seed=0):
 # GPU arm
 # ---------------------------------------------------------------------------
 
+def weight_copy(step, batch_index, n_batches, copies):
+    """The weight copy that token batch `batch_index` of step `step` reads:
+    the batches of all steps walk the copies in order, so a copy is read again
+    only after every other copy has been."""
+    return (step * n_batches + batch_index) % copies
+
+
 def make_layers(w, seed, device, copies):
     """Build the layer set once on the host, then `copies` device copies of
     the packed weights and LUTs (distinct buffers, so rotation defeats L2)."""
@@ -353,9 +366,17 @@ def run_ours(args, w, rank, world, device):
                 plan.append((li, T, op, u))
     step_units = sum(p[3] for p in plan)
 
-    def launch(li, T, op, set_idx):
+    # every (step, token batch) reads its own copy of the weights: consecutive
+    # batches of a step do not share a copy, and a copy comes back only after
+    # all the others (more than 3x L2 of index bytes) have been streamed
+    batch_pos = {T: bi for bi, T in enumerate(w["batches"])}
+
+    def copy_of(s, T):
+        return weight_copy(s, batch_pos[T], len(w["batches"]), copies)
+
+    def launch(li, T, op, s):
         L = layers[li]
-        packed, lut = L["sets"][set_idx % len(L["sets"])]
+        packed, lut = L["sets"][copy_of(s, T)]
         a = acts[(li, T)]
         if op == "fwd":
             sk.linear_fwd(packed, lut, bits, a["X"], a["task"], out=a["Y"])
@@ -533,7 +554,7 @@ def run_ours(args, w, rank, world, device):
                 for (li, T, op, u) in plan:
                     x = dev_in[(li, T)]
                     L = layers[li]
-                    packed, lut = L["sets"][(W + s) % len(L["sets"])]
+                    packed, lut = L["sets"][copy_of(W + s, T)]
                     tk = x.get("task")
                     out = dev_out[(li, T, op)]
                     if op == "fwd":
@@ -817,13 +838,7 @@ def main():
         return main_sketch(args, w, world, rank, local)
     unit, scale = fmt_units(w)
     pk = peaks()
-    config = {"workload": args.workload, "desc": w["desc"], "bits": w["bits"], "gpr": w["gpr"],
-              "tokens": list(w["batches"]), "ntask": w["ntask"], "layers": [list(s) for s in layer_shapes(w)],
-              "parallelism": ("single" if world == 1 else
-                              f"dp{world} (tokens per rank; LUT-gradient all-reduce)" if "dlut" in w["ops"]
-                              else f"replicas{world}"),
-              "l2": "weights rotate over copies totalling > 3x L2",
-              "layer_subset": _LAYER_SUBSET}
+    config = workload_config(args.workload, w, world)
 
     if args.impl == "reference":
         if rank != 0:
@@ -852,12 +867,47 @@ def main():
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     device = torch.device("cuda", torch.cuda.current_device())
-    res = run_ours(args, w, rank, world, device)
+    line = measure(args, args.workload, w, config, world, rank, device, pk)
+    if args.workload == "decode7b" and not args.no_train and _LAYER_SUBSET is None:
+        # the metric's second half: the fwd+bwd TFLOP/s of the 7B-shaped
+        # fine-tune step, measured in the same run on the same GPU(s)
+        torch.cuda.empty_cache()
+        tw = WORKLOADS[TRAIN_WORKLOAD]
+        tconfig = workload_config(TRAIN_WORKLOAD, tw, world)
+        train = measure(args, TRAIN_WORKLOAD, tw, tconfig, world, rank, device, pk)
+        if line is not None:
+            line["train"] = {k: train[k] for k in ("value", "unit", "ms_per_step", "steps", "warmup", "dtype",
+                                                   "config", "roofline", "gpu_launches", "clocks", "e2e",
+                                                   "cpu_baseline") if k in train}
+            line["train"]["metric"] = "fwd+bwd TFLOP/s (% bf16 peak), sketched linear: Y, dX and dLUT per layer"
+            line["train"]["higher_is_better"] = True
+            line["gpu_launches"] += train["gpu_launches"]
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return 0
+    print(json.dumps(line))
+    return 0
+
+
+def workload_config(name, w, world):
+    return {"workload": name, "desc": w["desc"], "bits": w["bits"], "gpr": w["gpr"],
+            "tokens": list(w["batches"]), "ntask": w["ntask"], "layers": [list(s) for s in layer_shapes(w)],
+            "parallelism": ("single" if world == 1 else
+                            f"dp{world} (tokens per rank; LUT-gradient all-reduce)" if "dlut" in w["ops"]
+                            else f"replicas{world}"),
+            "l2": "weights rotate over copies totalling > 3x L2; every (step, token batch) reads its own copy",
+            "layer_subset": _LAYER_SUBSET}
+
+
+def measure(args, name, w, config, world, rank, device, pk):
+    """Time one workload on the GPU arm; rank 0 gets the JSON line (others None)."""
+    import torch
+    unit, scale = fmt_units(w)
+    res = run_ours(args, w, rank, world, device)
+    if rank != 0:
+        return None
 
     # the dominant kernel: the kernel type (op, tokens) with the largest share of
     # the step; its achieved rate = its algorithmic units / its measured time
@@ -873,13 +923,13 @@ def main():
     if res["hbm_bound"]:
         achieved = units / (t_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
-                "frac": achieved / pk["hbm"], "traffic": traffic_per_launch(kname, args.workload, units / max(nl, 1)),
+                "frac": achieved / pk["hbm"], "traffic": traffic_per_launch(kname, name, units / max(nl, 1)),
                 "kernel": kname, "launches_per_step": nl, "share": t_ms / step_ms,
                 "peak_source": pk["source"] + " hbm_gbs (copy)"}
     else:
         achieved = units / (t_ms / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_sus"], "unit": "TFLOP/s",
-                "frac": achieved / pk["bf16_sus"], "traffic": traffic_per_launch(kname, args.workload, units / max(nl, 1)),
+                "frac": achieved / pk["bf16_sus"], "traffic": traffic_per_launch(kname, name, units / max(nl, 1)),
                 "kernel": kname, "launches_per_step": nl, "share": t_ms / step_ms,
                 "peak_source": pk["source"] + " bf16_tflops_sustained (a kernel timed inside a long step)"}
     if res["hbm_bound"] and kname == "decode_kernel" and w["bits"] == 4:
@@ -907,12 +957,11 @@ def main():
         e = res["e2e"]
         line["e2e"] = {"value": e["value"] / scale, "unit": unit, "h2d_bytes_per_step": e["h2d"],
                        "d2h_bytes_per_step": e["d2h"]}
-    if not args.no_cpu_baseline:
-        units, el, cores, done = cpu_baseline(w, budget_s=12.0, seed=args.seed)
+    if not args.no_cpu_baseline and world == 1:
+        units, el, cores, done = cpu_baseline(w, budget_s=12.0 if res["hbm_bound"] else 8.0, seed=args.seed)
         line["cpu_baseline"] = {"value": units / el / scale, "unit": unit, "cores": cores, "kind": "oracle",
                                 "sample": "; ".join(f"layer {li} T={T}" for li, T, _ in done)}
-    print(json.dumps(line))
-    return 0
+    return line
 
 
 if __name__ == "__main__":

@@ -351,48 +351,83 @@ def sketch_layer(theta: torch.Tensor, X: torch.Tensor, bits: int, gpr: int, damp
 
 
 class SketchedLinearFunction(torch.autograd.Function):
-    """Y = X Theta_hat^T with gradients for X and for the LUT values only."""
+    """Y = X Theta_hat^T with gradients for X and for the LUT values only.
+
+    `lut` is the trainable tensor that receives the LUT gradient; `lut16` holds
+    the fp16 tables the kernels read (the same tensor when `lut` is fp16, else
+    the round-to-nearest-even fp16 of an fp32 master).  The LUT gradient is
+    computed in fp32 and returned in `lut`'s dtype: an fp32 master gets it
+    unrounded."""
 
     @staticmethod
-    def forward(ctx, X, lut, packed, bits, task):
-        Y = linear_fwd(packed, lut, bits, X.contiguous(), task)
-        ctx.save_for_backward(X, lut, packed, task if task is not None else torch.empty(0))
+    def forward(ctx, X, lut, lut16, packed, bits, task):
+        Y = linear_fwd(packed, lut16, bits, X.contiguous(), task)
+        ctx.save_for_backward(X, lut16, packed, task if task is not None else torch.empty(0))
         ctx.bits = bits
         ctx.has_task = task is not None
+        ctx.lut_dtype = lut.dtype
         return Y
 
     @staticmethod
     def backward(ctx, dY):
-        X, lut, packed, task = ctx.saved_tensors
+        X, lut16, packed, task = ctx.saved_tensors
         task = task if ctx.has_task else None
         dY = dY.contiguous().to(torch.bfloat16)
         dX = dlut = None
         if ctx.needs_input_grad[0]:
-            dX = linear_bwd_input(packed, lut, ctx.bits, X.shape[1], dY, task)
+            dX = linear_bwd_input(packed, lut16, ctx.bits, X.shape[1], dY, task)
         if ctx.needs_input_grad[1]:
-            ntask, n, gpr, _ = lut.shape
-            dlut = linear_bwd_lut(packed, ctx.bits, gpr, X, dY, task, ntask).to(lut.dtype)
-        return dX, dlut, None, None, None
+            ntask, n, gpr, _ = lut16.shape
+            dlut = linear_bwd_lut(packed, ctx.bits, gpr, X, dY, task, ntask)
+            if dlut.dtype != ctx.lut_dtype:
+                dlut = dlut.to(ctx.lut_dtype)
+        return dX, dlut, None, None, None, None
 
 
 def sketched_linear(X: torch.Tensor, lut: torch.Tensor, packed: torch.Tensor, bits: int,
-                    task: Optional[torch.Tensor] = None) -> torch.Tensor:
-    return SketchedLinearFunction.apply(X, lut, packed, bits, task)
+                    task: Optional[torch.Tensor] = None, lut16: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Y = X Theta_hat^T as an autograd function of X and of the LUT values.
+
+    lut: fp32 master LUTs (their gradient stays fp32) or fp16 LUTs (their
+    gradient is rounded to fp16).  lut16: the fp16 tables of an fp32 master,
+    when the caller keeps them (else they are rounded from `lut` here)."""
+    if lut16 is None:
+        lut16 = lut if lut.dtype == torch.float16 else lut.detach().to(torch.float16)
+    return SketchedLinearFunction.apply(X, lut, lut16, packed, bits, task)
 
 
 class SketchedLinear(torch.nn.Module):
     """A linear layer (no bias) whose weight is the sketch Theta_hat: a frozen
-    packed index map (buffer) and trainable fp16 LUTs [ntask, n, gpr, 2**bits]
-    (parameter).  forward(X, task) takes bf16 activations [..., d]; task holds
-    one LUT-set id per token (int32), or None for set 0."""
+    packed index map (buffer), trainable fp32 master LUTs [ntask, n, gpr,
+    2**bits] (parameter `lut`, whose gradient is the library's fp32 LUT
+    gradient) and the fp16 tables the kernels read (buffer `lut16`, the
+    round-to-nearest-even of the master).  forward(X, task) takes bf16
+    activations [..., d]; task holds one LUT-set id per token (int32), or None
+    for set 0.
+
+    `lut16` follows the master: `adamw_step` / `sgd_step` update both in one
+    library call; any other in-place change of `lut` (a torch optimizer) is
+    noticed by its version counter and `lut16` is rounded again before the
+    next forward."""
 
     def __init__(self, packed: torch.Tensor, lut: torch.Tensor, bits: int, in_features: int):
         super().__init__()
         self.register_buffer("packed", packed)
-        self.lut = torch.nn.Parameter(lut)
+        self.lut = torch.nn.Parameter(lut.detach().to(torch.float32).contiguous())
+        self.register_buffer("lut16", lut.detach().to(torch.float16).contiguous())
         self.bits = bits
         self.in_features = in_features
         self.out_features = lut.shape[1]
+        self._synced = self._lut_state()
+
+    def _lut_state(self):
+        return (self.lut.data_ptr(), self.lut._version)
+
+    def _sync_lut16(self):
+        if self._lut_state() != self._synced:
+            with torch.no_grad():
+                self.lut16.copy_(self.lut)
+            self._synced = self._lut_state()
 
     @classmethod
     def from_dense(cls, weight: torch.Tensor, X_calib: torch.Tensor, bits: int, gpr: int, ntask: int = 1,
@@ -403,7 +438,21 @@ class SketchedLinear(torch.nn.Module):
         return cls(packed, lut.unsqueeze(0).repeat(ntask, 1, 1, 1).contiguous(), bits, weight.shape[1])
 
     def forward(self, X: torch.Tensor, task: Optional[torch.Tensor] = None) -> torch.Tensor:
+        self._sync_lut16()
         lead = X.shape[:-1]
         Y = sketched_linear(X.reshape(-1, self.in_features).to(torch.bfloat16).contiguous(), self.lut, self.packed,
-                            self.bits, task)
+                            self.bits, task, lut16=self.lut16)
         return Y.reshape(*lead, self.out_features)
+
+    def adamw_step(self, m: torch.Tensor, v: torch.Tensor, step: int, lr: float, beta1: float = 0.9,
+                   beta2: float = 0.999, eps: float = 1e-8, weight_decay: float = 0.0,
+                   counts: Optional[torch.Tensor] = None) -> None:
+        """One AdamW step of the master LUTs from their gradient; rewrites lut16."""
+        self._sync_lut16()
+        lut_adamw_(self.lut.data, m, v, self.lut.grad, self.bits, step, lr, beta1, beta2, eps, weight_decay,
+                   counts, self.lut16)
+
+    def sgd_step(self, lr: float, counts: Optional[torch.Tensor] = None) -> None:
+        """One SGD step of the master LUTs from their gradient; rewrites lut16."""
+        self._sync_lut16()
+        lut_sgd_(self.lut.data, self.lut.grad, self.bits, lr, counts, self.lut16)

@@ -77,3 +77,18 @@ def test_stale_traffic_reads_as_null(monkeypatch, tmp_path):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     kernel, workload = key.split("@")
     assert bench.traffic_per_launch(kernel, workload, recs[key]["algorithmic_units"]) is None
+
+
+def test_every_batch_reads_its_own_weight_copy():
+    """Decode: the T=1 and T=16 batches of a step, and consecutive steps, read
+    distinct copies; a copy returns only after all the others, which together
+    hold more than 3x L2 of index bytes."""
+    w = W["decode7b"]
+    weight_bytes = sum(n * d * w["bits"] // 8 for n, d in synth.LLAMA2_7B)
+    copies = max(2, int(-(-3 * bench.L2_BYTES // weight_bytes)) + 1)
+    nb = len(w["batches"])
+    seq = [bench.weight_copy(s, bi, nb, copies) for s in range(12) for bi in range(nb)]
+    for i in range(len(seq)):
+        window = seq[i:i + copies]
+        assert len(set(window)) == len(window)
+    assert (copies - 1) * weight_bytes > 3 * bench.L2_BYTES

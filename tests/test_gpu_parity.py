@@ -247,6 +247,20 @@ def test_autograd_function():
     gc.check_dlut(L2.grad.float().cpu().numpy()[0], ref, "lut.grad")
 
 
+def test_autograd_function_fp32_master_lut():
+    """An fp32 master LUT gets the library's fp32 LUT gradient unrounded
+    (1024 tokens, dY ~ N(0, 1e-2), the 2e-3 bounds)."""
+    sk = _sk()
+    c = synth.layer_case(7310, n=256, d=1024, bits=4, gpr=4, T=1024)
+    packed, lut, X, dY, task = gc.dev_case(c)
+    L32 = lut.float().requires_grad_(True)
+    Y = sk.sketched_linear(X, L32, packed, c.bits)
+    gc.check_fwd(c, Y.detach())
+    Y.backward(dY)
+    assert L32.grad.dtype == torch.float32
+    gc.check_dlut(L32.grad.cpu().numpy()[0], oracle.backward_lut(c.x, c.dy, c.idx, c.gpr, c.k), "fp32 lut.grad")
+
+
 # ---------------------------------------------------------------------------
 # full-size layers, sampled rows: LLaMA-2-7B decode (4-bit, 8 groups per row)
 # ---------------------------------------------------------------------------
