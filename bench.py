@@ -98,6 +98,9 @@ def parse():
                     help="comma-separated layer indices to run (a subset for profiling); default all")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-groups", choices=("block", "all", "layer"), default="block",
+                    help="decode forward calls: 'block' groups the projections that share an input "
+                         "(q/k/v, gate/up), 'all' one call for the seven, 'layer' one call per layer")
     ap.add_argument("--no-train", action="store_true",
                     help="with the default decode workload, skip the fine-tune block (the metric's fwd+bwd half)")
     ap.add_argument("--launch-events", choices=("groups", "on", "off"), default="groups",
@@ -147,10 +150,10 @@ def kernel_name(op, T, w):
     """The library kernel a launch of this kind runs (the dispatch rules of sk_api.cu)."""
     if op == "fwd":
         if w["ntask"] > 1:
-            return "decode_kernel" if (T == 1 and w["bits"] == 4) else "fwd_tc_kernel (routed)"
+            return "decode_group_kernel" if (T == 1 and w["bits"] == 4) else "fwd_tc_kernel (routed)"
         path = os.environ.get("SK_FWD_PATH", "")
         if w["bits"] == 4 and T <= 16 and path not in ("gemv", "tc"):
-            return "decode_kernel"
+            return "decode_group_kernel"
         if path == "gemv" or (T == 1 and path != "tc"):
             return "gemv_fwd_single_kernel"
         return "fwd_tc_kernel"
@@ -299,6 +302,26 @@ def cpu_baseline(w, budget_s=15.0, seed=0):
 # GPU arm
 # ---------------------------------------------------------------------------
 
+# A decoder block's projections in the order a block runs them; the members
+# of a group read the same input (q/k/v; gate/up), so a real block can issue
+# each group as one call.
+BLOCK_GROUPS = ((0, 1, 2), (3,), (4, 5), (6,))
+
+
+def decode_groups(w, how, nlayers):
+    """The forward groups of a decode workload (one library call each), or
+    None for per-layer calls: 'block' groups the layers that share an input in
+    a decoder block, 'all' issues the seven projections (independent inputs
+    here) as one call, 'layer' one call per layer."""
+    if not (is_hbm_bound(w) and w["ops"] == ("fwd",) and w["bits"] == 4 and w["ntask"] == 1) or how == "layer":
+        return None
+    if _LAYER_SUBSET is not None or nlayers != 7:
+        return [tuple(range(nlayers))] if how == "all" else None
+    if how == "all":
+        return [tuple(range(7))]
+    return [g for g in BLOCK_GROUPS]
+
+
 def weight_copy(step, batch_index, n_batches, copies):
     """The weight copy that token batch `batch_index` of step `step` reads:
     the batches of all steps walk the copies in order, so a copy is read again
@@ -337,6 +360,16 @@ def run_ours(args, w, rank, world, device):
     layers = make_layers(w, args.seed, device, copies)
     rng = synth.rng_for(10_000 + rank)
 
+    # how the forward launches are grouped (decode workloads): each group is
+    # one library call; layers of a group that read the same input in a
+    # decoder block (q/k/v, gate/up) share one X
+    groups = decode_groups(w, args.decode_groups, len(layers))
+    share_x = {}
+    for grp in groups or ():
+        for li in grp:
+            if args.decode_groups == "block":
+                share_x[li] = grp[0]
+
     # activations / gradients per (layer, batch)
     acts = {}
     for li, L in enumerate(layers):
@@ -344,6 +377,9 @@ def run_ours(args, w, rank, world, device):
             X = torch.from_numpy(synth.make_bf16(rng, (T, L["d"]), synth.X_STD).view(np.int16)).to(device).view(torch.bfloat16)
             dY = torch.from_numpy(synth.make_bf16(rng, (T, L["n"]), synth.DY_STD).view(np.int16)).to(device).view(torch.bfloat16)
             task = torch.from_numpy(synth.make_task(rng, T, ntask)).to(device) if ntask > 1 else None
+            if share_x.get(li, li) != li:
+                X = acts[(share_x[li], T)]["X"]
+                task = acts[(share_x[li], T)]["task"]
             outs = dict(Y=torch.empty((T, L["n"]), dtype=torch.bfloat16, device=device))
             if "dx" in w["ops"]:
                 outs["dX"] = torch.empty((T, L["d"]), dtype=torch.bfloat16, device=device)
@@ -351,10 +387,20 @@ def run_ours(args, w, rank, world, device):
                 outs["dl"] = torch.empty((ntask, L["n"], gpr, 1 << bits), dtype=torch.float32, device=device)
             acts[(li, T)] = dict(X=X, dY=dY, task=task, **outs)
 
-    # launch list of one step: (layer, T, op, units)
+    # launch list of one step: (layers, T, op, units); `layers` is a tuple of
+    # layer indices, several for a grouped forward
     hbm_bound = is_hbm_bound(w)
     plan = []
     for T in w["batches"]:
+        if groups is not None:
+            for grp in groups:
+                u = 0
+                for li in grp:
+                    a, L = acts[(li, T)], layers[li]
+                    present = ntask if a["task"] is None else int(torch.unique(a["task"]).numel())
+                    u += launch_bytes(L["n"], L["d"], bits, gpr, T, present)
+                plan.append((tuple(grp), T, "fwd", u))
+            continue
         for li, L in enumerate(layers):
             for op in w["ops"]:
                 if hbm_bound:
@@ -363,7 +409,7 @@ def run_ours(args, w, rank, world, device):
                     u = launch_bytes(L["n"], L["d"], bits, gpr, T, present)
                 else:
                     u = launch_flops(L["n"], L["d"], T, op)
-                plan.append((li, T, op, u))
+                plan.append(((li,), T, op, u))
     step_units = sum(p[3] for p in plan)
 
     # every (step, token batch) reads its own copy of the weights: consecutive
@@ -374,16 +420,30 @@ def run_ours(args, w, rank, world, device):
     def copy_of(s, T):
         return weight_copy(s, batch_pos[T], len(w["batches"]), copies)
 
-    def launch(li, T, op, s):
+    def call(members, T, op, s, X_of, task, out_of, dy_of=None):
+        """One library call of the plan: X_of(li), dy_of(li) and out_of(li)
+        give the tensors (device-resident or staged views)."""
+        dy_of = dy_of or (lambda li: acts[(li, T)]["dY"])
+        if len(members) > 1 or groups is not None:
+            ls = [(layers[li]["sets"][copy_of(s, T)][0], layers[li]["sets"][copy_of(s, T)][1], X_of(li))
+                  for li in members]
+            sk.linear_fwd_group(ls, bits, task, outs=[out_of(li) for li in members])
+            return
+        li = members[0]
         L = layers[li]
         packed, lut = L["sets"][copy_of(s, T)]
-        a = acts[(li, T)]
         if op == "fwd":
-            sk.linear_fwd(packed, lut, bits, a["X"], a["task"], out=a["Y"])
+            sk.linear_fwd(packed, lut, bits, X_of(li), task, out=out_of(li))
         elif op == "dx":
-            sk.linear_bwd_input(packed, lut, bits, L["d"], a["dY"], a["task"], out=a["dX"])
+            sk.linear_bwd_input(packed, lut, bits, L["d"], dy_of(li), task, out=out_of(li))
         else:
-            sk.linear_bwd_lut(packed, bits, gpr, a["X"], a["dY"], a["task"], ntask, out=a["dl"])
+            sk.linear_bwd_lut(packed, bits, gpr, X_of(li), dy_of(li), task, ntask, out=out_of(li))
+
+    out_key = {"fwd": "Y", "dx": "dX", "dlut": "dl"}
+
+    def launch(members, T, op, s):
+        call(members, T, op, s, lambda li: acts[(li, T)]["X"], acts[(members[0], T)]["task"],
+             lambda li: acts[(li, T)][out_key[op]])
 
     # data-parallel fine-tuning: every rank runs its own T tokens (weak
     # scaling) and the LUT gradients are summed over ranks, one all-reduce per
@@ -393,9 +453,10 @@ def run_ours(args, w, rank, world, device):
         from compressive_fine_tuning_b200 import dp
         reducer = dp.LutGradReducer()
 
-    def after(op, li, T):
+    def after(op, members, T):
         if reducer is not None and op == "dlut":
-            reducer.submit(acts[(li, T)]["dl"])
+            for li in members:
+                reducer.submit(acts[(li, T)]["dl"])
 
     def end_step():
         if reducer is not None:
@@ -501,24 +562,21 @@ def run_ours(args, w, rank, world, device):
             return (nbytes + 255) // 256 * 256
 
         needs = {"fwd": ("X", "task"), "dx": ("dY", "task"), "dlut": ("X", "dY", "task")}
-        used = {}
-        for (li, T, op, u) in plan:
-            used.setdefault((li, T), set()).update(needs[op])
+        # staging offsets per distinct input tensor (layers of a group may share
+        # one X) and per output
         in_views, out_views, in_off, out_off = {}, {}, 0, 0
-        for (li, T, op, u) in plan:
-            a = acts[(li, T)]
-            if (li, T) not in in_views:
-                ent = {}
-                for name in ("X", "dY", "task"):
+        for (members, T, op, u) in plan:
+            for li in members:
+                a = acts[(li, T)]
+                for name in needs[op]:
                     t = a[name]
-                    if t is None or name not in used[(li, T)]:
+                    if t is None or id(t) in in_views:
                         continue
-                    ent[name] = (in_off, t)
+                    in_views[id(t)] = (in_off, t)
                     in_off += slab(t.numel() * t.element_size())
-                in_views[(li, T)] = ent
-            key = {"fwd": "Y", "dx": "dX", "dlut": "dl"}[op]
-            out_views[(li, T, op)] = (out_off, a[key])
-            out_off += slab(a[key].numel() * a[key].element_size())
+                out = a[out_key[op]]
+                out_views[(li, T, op)] = (out_off, out)
+                out_off += slab(out.numel() * out.element_size())
         hin = torch.empty(in_off, dtype=torch.uint8, pin_memory=True)
         din = torch.empty(in_off, dtype=torch.uint8, device=device)
         hout = torch.empty(out_off, dtype=torch.uint8, pin_memory=True)
@@ -528,13 +586,17 @@ def run_ours(args, w, rank, world, device):
             nb = like.numel() * like.element_size()
             return buf[off:off + nb].view(like.dtype).view(like.shape)
 
-        for (li, T), ent in in_views.items():
-            for name, (off, t) in ent.items():
-                view(hin, off, t).copy_(t.cpu())
-        dev_in = {key: {name: view(din, off, t) for name, (off, t) in ent.items()} for key, ent in in_views.items()}
+        for key, (off, t) in in_views.items():
+            view(hin, off, t).copy_(t.cpu())
+        dev_in = {key: view(din, off, t) for key, (off, t) in in_views.items()}
         dev_out = {key: view(dout, off, t) for key, (off, t) in out_views.items()}
+
+        def staged(li, T, name):
+            t = acts[(li, T)][name]
+            return None if t is None else dev_in[id(t)]
+
         # bytes that cross the bus per step: each input once, each result once
-        h2d = sum(t.numel() * t.element_size() for ent in in_views.values() for (_, t) in ent.values())
+        h2d = sum(t.numel() * t.element_size() for (_, t) in in_views.values())
         d2h = sum(t.numel() * t.element_size() for (_, t) in out_views.values())
         # transfers are issued in pieces of at most 64 MiB (one piece for a
         # decode step)
@@ -547,24 +609,20 @@ def run_ours(args, w, rank, world, device):
             dist.barrier()
         torch.cuda.synchronize(device)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        staged_dy = {}
         with torch.cuda.stream(stream):
             e0.record(stream)
             for s in range(K):
                 copy_in_pieces(din, hin)
-                for (li, T, op, u) in plan:
-                    x = dev_in[(li, T)]
-                    L = layers[li]
-                    packed, lut = L["sets"][copy_of(W + s, T)]
-                    tk = x.get("task")
-                    out = dev_out[(li, T, op)]
-                    if op == "fwd":
-                        sk.linear_fwd(packed, lut, bits, x["X"], tk, out=out)
-                    elif op == "dx":
-                        sk.linear_bwd_input(packed, lut, bits, L["d"], x["dY"], tk, out=out)
-                    else:
-                        sk.linear_bwd_lut(packed, bits, gpr, x["X"], x["dY"], tk, ntask, out=out)
+                for (members, T, op, u) in plan:
+                    if "dY" in needs[op]:
+                        for li in members:
+                            staged_dy[li] = staged(li, T, "dY")
+                    call(members, T, op, W + s, lambda li: staged(li, T, "X"), staged(members[0], T, "task"),
+                         lambda li: dev_out[(li, T, op)], dy_of=lambda li: staged_dy[li])
                     if reducer is not None and op == "dlut":
-                        reducer.submit(out)
+                        for li in members:
+                            reducer.submit(dev_out[(li, T, op)])
                         reducer.wait()
                 copy_in_pieces(hout, dout)
             e1.record(stream)
@@ -932,13 +990,14 @@ def measure(args, name, w, config, world, rank, device, pk):
                 "frac": achieved / pk["bf16_sus"], "traffic": traffic_per_launch(kname, name, units / max(nl, 1)),
                 "kernel": kname, "launches_per_step": nl, "share": t_ms / step_ms,
                 "peak_source": pk["source"] + " bf16_tflops_sustained (a kernel timed inside a long step)"}
-    if res["hbm_bound"] and kname == "decode_kernel" and w["bits"] == 4:
+    if res["hbm_bound"] and kname == "decode_group_kernel" and w["bits"] == 4:
         # The decode kernel is bound by the integer pipe, not by HBM: every 4-bit
         # weight costs 2.25 integer-ALU lane operations at least (16 byte permutes
         # and 2 masks per eight weights), and the integer pipe issues 64 lanes per
         # cycle per SM on this GPU (measured).  Reported beside the HBM roofline.
         shapes = layer_shapes(w)
-        lookups = sum(shapes[li][0] * shapes[li][1] for (li, T_, op_, u_) in res["plan"] if (op_, T_) == dom)
+        lookups = sum(shapes[li][0] * shapes[li][1] for (members, T_, op_, u_) in res["plan"] if (op_, T_) == dom
+                      for li in members)
         mhz = (res["clocks"] or {}).get("sm_mhz") or 1965.0
         ops = lookups * ALU_OPS_PER_4BIT_WEIGHT / (t_ms / 1e3)
         alu_peak = torch.cuda.get_device_properties(device).multi_processor_count * INT_LANES_PER_SM * mhz * 1e6

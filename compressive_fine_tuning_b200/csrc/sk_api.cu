@@ -323,6 +323,66 @@ sk_status sk_linear_fwd(const void* packed, const uint16_t* lut, int bits, int g
   return e == cudaSuccess ? ok() : cuda_fail(e, "forward kernel launch");
 }
 
+sk_status sk_linear_fwd_group(const sk_layer* layers, int nlayers, int bits, int64_t T, const int32_t* task,
+                              int ntask, sk_stream_t stream) {
+  g_last_error.clear();
+  if (nlayers < 1 || nlayers > SK_MAX_GROUP_LAYERS)
+    return fail(SK_ERR_INVALID_ARG, "nlayers must be in [1, %d] (got %d)", SK_MAX_GROUP_LAYERS, nlayers);
+  if (layers == nullptr) return fail(SK_ERR_INVALID_ARG, "null pointer");
+  for (int l = 0; l < nlayers; ++l) {
+    const sk_layer& L = layers[l];
+    sk_status st = check_shape(bits, L.gpr, L.n, L.d, T, ntask);
+    if (st != SK_OK) return fail(st, "layer %d: %s", l, g_last_error.c_str());
+    if (T == 0) continue;
+    st = check_layer_buffers(L.packed, L.lut, true, bits, L.gpr, L.n, L.d, T, task, ntask, L.X, (size_t)(T * L.d * 2),
+                             nullptr, 0, L.Y, (size_t)(T * L.n * 2));
+    if (st != SK_OK) return fail(st, "layer %d: %s", l, g_last_error.c_str());
+  }
+  if (T == 0) return ok();
+  // the layers run side by side: no output may overlap another layer's buffers
+  for (int a = 0; a < nlayers; ++a) {
+    const sk_layer& A = layers[a];
+    const size_t ya = (size_t)(T * A.n * 2);
+    for (int b = 0; b < nlayers; ++b) {
+      if (a == b) continue;
+      const sk_layer& B = layers[b];
+      const size_t lb = (size_t)ntask * B.n * B.gpr * (1u << bits) * 2;
+      if (overlaps(A.Y, ya, B.Y, (size_t)(T * B.n * 2)) || overlaps(A.Y, ya, B.X, (size_t)(T * B.d * 2)) ||
+          overlaps(A.Y, ya, B.packed, sk_packed_bytes(B.n, B.d, bits)) || overlaps(A.Y, ya, B.lut, lb))
+        return fail(SK_ERR_INVALID_ARG, "the output of layer %d overlaps a buffer of layer %d", a, b);
+    }
+  }
+  unsigned int* check = nullptr;
+  sk_status st = device_state(&check);
+  if (st != SK_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  sk::DecodeLayer D[SK_MAX_GROUP_LAYERS];
+  for (int l = 0; l < nlayers; ++l) {
+    const sk_layer& L = layers[l];
+    D[l].packed = static_cast<const uint8_t*>(L.packed);
+    D[l].row_bytes = (int64_t)row_bytes(L.d, bits);
+    D[l].lut = L.lut;
+    D[l].gpr = L.gpr;
+    D[l].n = L.n;
+    D[l].d = L.d;
+    D[l].X = L.X;
+    D[l].Y = L.Y;
+  }
+  const int forced = env_path("SK_FWD_PATH");
+  if (bits == 4 && forced != 1 && forced != 2 && sk::decode_group_supported(D, nlayers, (int)T, task, ntask)) {
+    cudaError_t e = sk::launch_decode_group(D, nlayers, (int)T, task, ntask, check, s);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "grouped decode kernel launch");
+  }
+  // otherwise one forward per layer, in order (no workspace: a batch with
+  // several LUT sets runs on the CUDA-core kernel)
+  for (int l = 0; l < nlayers; ++l) {
+    const sk_layer& L = layers[l];
+    st = sk_linear_fwd(L.packed, L.lut, bits, L.gpr, L.n, L.d, L.X, T, task, ntask, L.Y, nullptr, 0, stream);
+    if (st != SK_OK) return st;
+  }
+  return ok();
+}
+
 sk_status sk_linear_bwd_input(const void* packed, const uint16_t* lut, int bits, int gpr, int64_t n, int64_t d,
                               const uint16_t* dY, int64_t T, const int32_t* task, int ntask, uint16_t* dX,
                               void* workspace, size_t workspace_bytes, sk_stream_t stream) {

@@ -355,6 +355,20 @@ cudaError_t launch_gemv_fwd(const Problem& p, const uint16_t* X, uint16_t* Y, cu
 // Decode forward (4-bit, single LUT set, 1 <= T <= 16, d >= 256) on mma.sync.
 bool decode_fwd_supported(const Problem& p);
 cudaError_t launch_decode_fwd(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStream_t s);
+// The same for a group of layers with one token batch size, in one launch.
+constexpr int kMaxDecodeGroup = 8;
+struct DecodeLayer {
+  const uint8_t* packed;   // [n][row_bytes], 4-bit
+  int64_t row_bytes;
+  const uint16_t* lut;     // fp16 [ntask][n][gpr][16]
+  int gpr;
+  int64_t n, d;
+  const uint16_t* X;       // bf16 [T][d]
+  uint16_t* Y;             // bf16 [T][n]
+};
+bool decode_group_supported(const DecodeLayer* layers, int nl, int T, const int32_t* task, int ntask);
+cudaError_t launch_decode_group(const DecodeLayer* layers, int nl, int T, const int32_t* task, int ntask,
+                                unsigned int* check, cudaStream_t s);
 cudaError_t launch_fwd_tc(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStream_t s);
 cudaError_t launch_dx_tc(const Problem& p, const uint16_t* dY, uint16_t* dX, cudaStream_t s);
 // dX for a batch with several LUT sets: tokens routed by task (workspace of

@@ -25,11 +25,21 @@ SK_CHECK_LUT_ORDER = 16
 
 EXPORTED = (
     "sk_abi_version", "sk_status_string", "sk_last_error", "sk_packed_row_bytes", "sk_packed_bytes",
-    "sk_pack", "sk_unpack", "sk_dequant", "sk_workspace_bytes", "sk_linear_fwd", "sk_linear_bwd_input",
+    "sk_pack", "sk_unpack", "sk_dequant", "sk_workspace_bytes", "sk_linear_fwd", "sk_linear_fwd_group",
+    "sk_linear_bwd_input",
     "sk_linear_bwd_lut", "sk_linear_bwd_lut_noalloc", "sk_bin_counts", "sk_lut_adamw", "sk_lut_sgd",
     "sk_device_check", "sk_inverse_factor_workspace_bytes", "sk_sketch_round_workspace_bytes", "sk_gram",
     "sk_inverse_factor", "sk_lloyd", "sk_sketch_round",
 )
+
+
+SK_MAX_GROUP_LAYERS = 8
+
+
+class _Layer(ctypes.Structure):
+    """sk_layer of sk.h: one layer of a grouped forward."""
+    _fields_ = [("packed", ctypes.c_void_p), ("lut", ctypes.c_void_p), ("gpr", ctypes.c_int),
+                ("n", ctypes.c_int64), ("d", ctypes.c_int64), ("X", ctypes.c_void_p), ("Y", ctypes.c_void_p)]
 
 
 class SketchError(RuntimeError):
@@ -55,6 +65,7 @@ def _load() -> ctypes.CDLL:
         "sk_dequant": ([vp, vp, i32, i32, i64, i64, i32, i32, vp, vp], i32),
         "sk_workspace_bytes": ([i32, i64, i64, i32, i32, i64, i32], sz),
         "sk_linear_fwd": ([vp, vp, i32, i32, i64, i64, vp, i64, vp, i32, vp, vp, sz, vp], i32),
+        "sk_linear_fwd_group": ([ctypes.POINTER(_Layer), i32, i32, i64, vp, i32, vp], i32),
         "sk_linear_bwd_input": ([vp, vp, i32, i32, i64, i64, vp, i64, vp, i32, vp, vp, sz, vp], i32),
         "sk_linear_bwd_lut": ([vp, i32, i32, i64, i64, vp, vp, i64, vp, i32, vp, i32, vp, sz, vp], i32),
         "sk_linear_bwd_lut_noalloc": ([vp, i32, i32, i64, i64, vp, vp, i64, vp, i32, vp, i32, vp], i32),
@@ -185,6 +196,33 @@ def linear_fwd(packed: torch.Tensor, lut: torch.Tensor, bits: int, X: torch.Tens
     _check(lib.sk_linear_fwd(_ptr(packed), _ptr(lut), bits, gpr, n, d, _ptr(X), T, _ptr(task), ntask,
                              _ptr(out), _ptr(ws), nb, _stream(X.device)))
     return out
+
+
+def linear_fwd_group(layers, bits: int, task: Optional[torch.Tensor] = None, outs=None):
+    """Y_l = X_l Theta_hat_l^T for a list of layers (packed, lut, X) that see the
+    same number of tokens, in one library call (one launch at decode sizes).
+    Returns the list of Y_l; `outs` may give them."""
+    if not 1 <= len(layers) <= SK_MAX_GROUP_LAYERS:
+        raise ValueError(f"1 to {SK_MAX_GROUP_LAYERS} layers per group")
+    arr = (_Layer * len(layers))()
+    T = None
+    ntask = None
+    ys = []
+    for i, (packed, lut, X) in enumerate(layers):
+        nt, n, gpr = _lut_shape(lut, bits)
+        _need(X, torch.bfloat16, "X", 2)
+        _need(packed, torch.uint8, "packed")
+        if T is None:
+            T, ntask = X.shape[0], nt
+        elif X.shape[0] != T or nt != ntask:
+            raise ValueError("every layer of a group must see the same tokens and LUT sets")
+        Y = outs[i] if outs is not None else torch.empty((T, n), dtype=torch.bfloat16, device=X.device)
+        _need(Y, torch.bfloat16, "out", 2)
+        ys.append(Y)
+        arr[i] = _Layer(packed.data_ptr(), lut.data_ptr(), gpr, n, X.shape[1], X.data_ptr(), Y.data_ptr())
+    task = _task_arg(task, T)
+    _check(lib.sk_linear_fwd_group(arr, len(layers), bits, T, _ptr(task), ntask, _stream(layers[0][2].device)))
+    return ys
 
 
 def linear_bwd_input(packed: torch.Tensor, lut: torch.Tensor, bits: int, d: int, dY: torch.Tensor,

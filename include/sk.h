@@ -154,6 +154,34 @@ sk_status sk_linear_fwd(const void* packed, const uint16_t* lut, int bits, int g
                         void* workspace, size_t workspace_bytes, sk_stream_t stream);
 
 /*
+ * sk_linear_fwd_group: the forward of several layers that see the same number
+ * of tokens, in one call: for every layer l, Y_l = X_l Theta_hat_l^T exactly as
+ * sk_linear_fwd computes it (same precision, same LUT-set rule).  Typical use:
+ * the projections of a decoder block at decode batch sizes, where each layer
+ * alone is too small to keep the GPU busy across a launch boundary.
+ *
+ * With 4-bit indices, 1 <= T <= 16 and one LUT set per call (or several sets
+ * and a single token) the layers run in one launch, spread over the SMs in
+ * proportion to their size; otherwise the call runs sk_linear_fwd for each
+ * layer in order, without a workspace.  Layers may share an input X (the
+ * q/k/v or gate/up projections of a block); no layer's Y may overlap any
+ * buffer of any layer.  `task` and `ntask` apply to every layer.  At most
+ * SK_MAX_GROUP_LAYERS layers; the array itself is host memory and is not
+ * kept after the call returns.
+ */
+#define SK_MAX_GROUP_LAYERS 8
+typedef struct {
+  const void* packed;      /* device, packed index map of the layer */
+  const uint16_t* lut;     /* device fp16 [ntask][n][gpr][2^bits]     */
+  int gpr;
+  int64_t n, d;
+  const uint16_t* X;       /* device bf16 [T][d]                       */
+  uint16_t* Y;             /* device bf16 [T][n]                       */
+} sk_layer;
+sk_status sk_linear_fwd_group(const sk_layer* layers, int nlayers, int bits, int64_t T,
+                              const int32_t* task, int ntask, sk_stream_t stream);
+
+/*
  * sk_linear_bwd_input: dX = dY Theta_hat (chain rule through the frozen
  * sketch; the layer has to pass gradients back to earlier layers).  Same
  * precision rules as sk_linear_fwd.

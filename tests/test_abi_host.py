@@ -293,3 +293,26 @@ def test_noalloc_rejects_layers_beyond_its_scratch():
     st, msg = r.stdout.strip().split(" ", 1)
     assert int(st) == SK_ERR_INVALID_ARG
     assert "scratch" in msg
+
+
+def test_group_validation():
+    """The grouped forward checks every layer and the overlaps between layers
+    on the host, before touching a device."""
+    L = sk.lib
+    mk = lambda p, lut, X, Y, n=256, d=512, gpr=1: sk._Layer(p, lut, gpr, n, d, X, Y)
+    base = 0x10000000
+    a = mk(base, base + 0x1000000, base + 0x2000000, base + 0x3000000)
+    b = mk(base + 0x4000000, base + 0x5000000, base + 0x6000000, base + 0x7000000)
+    arr = (sk._Layer * 9)(*([a, b] * 4 + [a]))
+    assert L.sk_linear_fwd_group(arr, 0, 4, 4, None, 1, None) == SK_ERR_INVALID_ARG
+    assert L.sk_linear_fwd_group(arr, 9, 4, 4, None, 1, None) == SK_ERR_INVALID_ARG
+    assert L.sk_linear_fwd_group(None, 1, 4, 4, None, 1, None) == SK_ERR_INVALID_ARG
+    bad = (sk._Layer * 2)(a, mk(base + 0x4000000, base + 0x5000000, base + 0x6000000, base + 0x3000000 + 16))
+    assert L.sk_linear_fwd_group(bad, 2, 4, 4, None, 1, None) == SK_ERR_INVALID_ARG   # outputs overlap
+    assert b"overlaps" in L.sk_last_error()
+    reads = (sk._Layer * 2)(a, mk(base + 0x4000000, base + 0x5000000, base + 0x3000000, base + 0x7000000))
+    assert L.sk_linear_fwd_group(reads, 2, 4, 4, None, 1, None) == SK_ERR_INVALID_ARG  # Y of one is X of another
+    shape = (sk._Layer * 2)(a, mk(base + 0x4000000, base + 0x5000000, base + 0x6000000, base + 0x7000000, d=48))
+    assert L.sk_linear_fwd_group(shape, 2, 4, 4, None, 1, None) == SK_ERR_INVALID_ARG
+    assert b"layer 1" in L.sk_last_error()
+    assert L.sk_linear_fwd_group(arr, 2, 4, 0, None, 1, None) == SK_OK                 # no tokens: nothing to do

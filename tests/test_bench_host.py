@@ -31,12 +31,12 @@ def test_training_flops_are_three_products():
 
 
 @pytest.mark.parametrize("op,T,workload,name", [
-    ("fwd", 1, "decode7b", "decode_kernel"),
-    ("fwd", 16, "decode7b", "decode_kernel"),
+    ("fwd", 1, "decode7b", "decode_group_kernel"),
+    ("fwd", 16, "decode7b", "decode_group_kernel"),
     ("fwd", 8192, "finetune7b", "fwd_tc_kernel"),
     ("dx", 8192, "finetune7b", "dx_tc_kernel"),
     ("dlut", 8192, "finetune7b_mt", "dlut_tc_kernel (routed)"),
-    ("fwd", 1, "serve70b_decode", "decode_kernel"),
+    ("fwd", 1, "serve70b_decode", "decode_group_kernel"),
     ("fwd", 64, "serve70b_decode", "fwd_tc_kernel (routed)"),
 ])
 def test_kernel_attribution(op, T, workload, name, monkeypatch):

@@ -122,3 +122,80 @@ def test_decode_single_token_bad_task_zeroes_and_flags():
     Y = sk.linear_fwd(packed, lut, 4, X, task)
     assert sk.device_check(clear=True) & sk.SK_CHECK_TASK_RANGE
     assert not Y.float().abs().any()
+
+
+# ---------------------------------------------------------------------------
+# several layers in one call (sk_linear_fwd_group)
+# ---------------------------------------------------------------------------
+
+def _shared_x(c, src):
+    """The case `c` with the activations of `src` (layers that read one input)."""
+    return synth.LayerCase(c.n, c.d, c.bits, c.gpr, src.T, c.ntask, c.idx, c.lut, src.x_bits, c.dy_bits, src.task)
+
+
+@pytest.mark.parametrize("T", [1, 5, 9, 16])
+def test_decode_group_matches_oracle(T):
+    """Mixed widths, ragged row tiles, groups that straddle stages, 32-column
+    groups and two layers that share one input, in one launch: every layer's
+    Y against the oracle."""
+    from compressive_fine_tuning_b200 import sk
+    shapes = [(264, 256, 1), (2376, 2816, 2), (96, 512, 16), (4104, 4096, 8), (1032, 4096, 8)]
+    cases = [synth.layer_case(36000 + 10 * i + T, n=n, d=d, bits=4, gpr=g, T=T) for i, (n, d, g) in enumerate(shapes)]
+    cases[4] = _shared_x(cases[4], cases[3])
+    dev = [gc.dev_case(c) for c in cases]
+    Xs = [dv[2] for dv in dev]
+    Xs[4] = Xs[3]
+    ys = sk.linear_fwd_group([(dv[0], dv[1], x) for dv, x in zip(dev, Xs)], 4)
+    torch.cuda.synchronize()
+    for c, y in zip(cases, ys):
+        gc.check_fwd(c, y)
+    assert sk.device_check() == 0
+    # the same call twice gives the same bits
+    ys2 = sk.linear_fwd_group([(dv[0], dv[1], x) for dv, x in zip(dev, Xs)], 4)
+    assert all(torch.equal(a, b) for a, b in zip(ys, ys2))
+
+
+@pytest.mark.parametrize("T", [1, 16])
+def test_decode_group_llama7b_block_sampled(T):
+    """The seven LLaMA-2-7B projections (4-bit, 8 groups per row) as one group,
+    q/k/v and gate/up each sharing an input: 96 sampled rows per layer."""
+    from compressive_fine_tuning_b200 import sk
+    cases = [synth.layer_case(37000 + 10 * i + T, n=n, d=d, bits=4, gpr=8, T=T)
+             for i, (n, d) in enumerate(synth.LLAMA2_7B)]
+    for i, src in ((1, 0), (2, 0), (5, 4)):
+        cases[i] = _shared_x(cases[i], cases[src])
+    dev = [gc.dev_case(c) for c in cases]
+    xs = [dev[{1: 0, 2: 0, 5: 4}.get(i, i)][2] for i in range(7)]
+    ys = sk.linear_fwd_group([(dv[0], dv[1], x) for dv, x in zip(dev, xs)], 4)
+    torch.cuda.synchronize()
+    assert sk.device_check() == 0
+    for i, (c, y) in enumerate(zip(cases, ys)):
+        rows = np.sort(synth.rng_for(37100 + i).choice(c.n, size=96, replace=False))
+        gc.check_fwd(c, y, rows=rows)
+
+
+def test_decode_group_single_token_multitask():
+    """One token with a task id over a group: every layer uses that set."""
+    from compressive_fine_tuning_b200 import sk
+    cases = [synth.layer_case(38000 + i, n=n, d=d, bits=4, gpr=4, T=1, ntask=8, with_task=True)
+             for i, (n, d) in enumerate([(1024, 2048), (512, 4096), (2048, 1024)])]
+    for c in cases:
+        c.task[:] = 6
+    dev = [gc.dev_case(c) for c in cases]
+    ys = sk.linear_fwd_group([(dv[0], dv[1], dv[2]) for dv in dev], 4, task=dev[0][4])
+    torch.cuda.synchronize()
+    for c, y in zip(cases, ys):
+        gc.check_fwd(c, y)
+    assert sk.device_check() == 0
+
+
+def test_group_outside_the_decode_kernel_runs_per_layer():
+    """2-bit layers at 64 tokens are not decode work: the group call runs the
+    layers one by one on their own kernels, with the same results."""
+    from compressive_fine_tuning_b200 import sk
+    cases = [synth.layer_case(39000 + i, n=n, d=d, bits=2, gpr=2, T=64) for i, (n, d) in enumerate([(256, 512), (136, 1024)])]
+    dev = [gc.dev_case(c) for c in cases]
+    ys = sk.linear_fwd_group([(dv[0], dv[1], dv[2]) for dv in dev], 2)
+    torch.cuda.synchronize()
+    for c, y in zip(cases, ys):
+        gc.check_fwd(c, y)
