@@ -4,7 +4,11 @@
 Default workload: LLaMA-2-7B-shaped decode (the seven layer shapes q/k/v/o
 4096x4096, gate/up 11008x4096, down 4096x11008; 4-bit indices, 8 groups per
 row, fp16 LUTs; X bf16 N(0,1) at 1 and at 16 tokens).  One step = the seven
-layers at T=1 followed by the seven layers at T=16, i.e. 14 forward launches.
+layers at T=1 followed by the seven layers at T=16.  Their inputs are
+independent activations, so by default each token count's seven layers are
+one grouped call (sk_linear_fwd_group, one launch); --decode-groups block
+groups only the layers that share an input in a decoder block, layer makes
+one call per layer.
 The metric is algorithmic bytes per second (packed indices + LUTs +
 activations in + outputs out), the LUT-GEMV's HBM roofline quantity.
 
@@ -98,9 +102,11 @@ def parse():
                     help="comma-separated layer indices to run (a subset for profiling); default all")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--decode-groups", choices=("block", "all", "layer"), default="block",
-                    help="decode forward calls: 'block' groups the projections that share an input "
-                         "(q/k/v, gate/up), 'all' one call for the seven, 'layer' one call per layer")
+    ap.add_argument("--decode-groups", choices=("block", "all", "layer"), default="all",
+                    help="decode forward calls: 'all' one grouped call for the seven projections of a "
+                         "token count (their inputs are independent here), 'block' groups only the "
+                         "projections that share an input in a decoder block (q/k/v, gate/up), 'layer' "
+                         "one call per layer")
     ap.add_argument("--no-train", action="store_true",
                     help="with the default decode workload, skip the fine-tune block (the metric's fwd+bwd half)")
     ap.add_argument("--launch-events", choices=("groups", "on", "off"), default="groups",
@@ -150,7 +156,7 @@ def kernel_name(op, T, w):
     """The library kernel a launch of this kind runs (the dispatch rules of sk_api.cu)."""
     if op == "fwd":
         if w["ntask"] > 1:
-            return "decode_group_kernel" if (T == 1 and w["bits"] == 4) else "fwd_tc_kernel (routed)"
+            return "decode_group_kernel" if (w["bits"] == 4 and T == 1) else "fwd_tc_kernel (routed)"
         path = os.environ.get("SK_FWD_PATH", "")
         if w["bits"] == 4 and T <= 16 and path not in ("gemv", "tc"):
             return "decode_group_kernel"
@@ -363,9 +369,9 @@ def run_ours(args, w, rank, world, device):
     # how the forward launches are grouped (decode workloads): each group is
     # one library call; layers of a group that read the same input in a
     # decoder block (q/k/v, gate/up) share one X
-    groups = decode_groups(w, args.decode_groups, len(layers))
+    fwd_groups = decode_groups(w, args.decode_groups, len(layers))
     share_x = {}
-    for grp in groups or ():
+    for grp in fwd_groups or ():
         for li in grp:
             if args.decode_groups == "block":
                 share_x[li] = grp[0]
@@ -392,8 +398,8 @@ def run_ours(args, w, rank, world, device):
     hbm_bound = is_hbm_bound(w)
     plan = []
     for T in w["batches"]:
-        if groups is not None:
-            for grp in groups:
+        if fwd_groups is not None:
+            for grp in fwd_groups:
                 u = 0
                 for li in grp:
                     a, L = acts[(li, T)], layers[li]
@@ -411,6 +417,15 @@ def run_ours(args, w, rank, world, device):
                     u = launch_flops(L["n"], L["d"], T, op)
                 plan.append(((li,), T, op, u))
     step_units = sum(p[3] for p in plan)
+    # LUT lookups of each forward launch: every weight once per LUT set present
+    plan_lookups = []
+    for (members, T, op, u) in plan:
+        lk = 0
+        for li in members:
+            a, L = acts[(li, T)], layers[li]
+            present = 1 if a["task"] is None else int(torch.unique(a["task"]).numel())
+            lk += L["n"] * L["d"] * present
+        plan_lookups.append(lk if op == "fwd" else 0)
 
     # every (step, token batch) reads its own copy of the weights: consecutive
     # batches of a step do not share a copy, and a copy comes back only after
@@ -424,7 +439,7 @@ def run_ours(args, w, rank, world, device):
         """One library call of the plan: X_of(li), dy_of(li) and out_of(li)
         give the tensors (device-resident or staged views)."""
         dy_of = dy_of or (lambda li: acts[(li, T)]["dY"])
-        if len(members) > 1 or groups is not None:
+        if len(members) > 1 or fwd_groups is not None:
             ls = [(layers[li]["sets"][copy_of(s, T)][0], layers[li]["sets"][copy_of(s, T)][1], X_of(li))
                   for li in members]
             sk.linear_fwd_group(ls, bits, task, outs=[out_of(li) for li in members])
@@ -550,7 +565,7 @@ def run_ours(args, w, rank, world, device):
         groups.append((kinds[0], step_units, ms / K, len(plan)))
     total_units = step_units * K * world
     value = total_units / (ms / 1e3)
-    res = dict(ms=ms, value=value, plan=plan, groups=groups, step_units=step_units,
+    res = dict(ms=ms, value=value, plan=plan, lookups=plan_lookups, groups=groups, step_units=step_units,
                hbm_bound=hbm_bound, clocks=clocks, copies=copies, weight_bytes=weight_bytes)
 
     # end-to-end through the public API with host buffers (one rank's view)
@@ -990,14 +1005,13 @@ def measure(args, name, w, config, world, rank, device, pk):
                 "frac": achieved / pk["bf16_sus"], "traffic": traffic_per_launch(kname, name, units / max(nl, 1)),
                 "kernel": kname, "launches_per_step": nl, "share": t_ms / step_ms,
                 "peak_source": pk["source"] + " bf16_tflops_sustained (a kernel timed inside a long step)"}
-    if res["hbm_bound"] and kname == "decode_group_kernel" and w["bits"] == 4:
+    if res["hbm_bound"] and kname.startswith("decode_group_kernel") and w["bits"] == 4:
         # The decode kernel is bound by the integer pipe, not by HBM: every 4-bit
-        # weight costs 2.25 integer-ALU lane operations at least (16 byte permutes
+        # lookup costs 2.25 integer-ALU lane operations at least (16 byte permutes
         # and 2 masks per eight weights), and the integer pipe issues 64 lanes per
-        # cycle per SM on this GPU (measured).  Reported beside the HBM roofline.
-        shapes = layer_shapes(w)
-        lookups = sum(shapes[li][0] * shapes[li][1] for (members, T_, op_, u_) in res["plan"] if (op_, T_) == dom
-                      for li in members)
+        # cycle per SM on this GPU (measured).  A weight is looked up once per
+        # LUT set present in the batch.  Reported beside the HBM roofline.
+        lookups = sum(lk for (members, T_, op_, u_), lk in zip(res["plan"], res["lookups"]) if (op_, T_) == dom)
         mhz = (res["clocks"] or {}).get("sm_mhz") or 1965.0
         ops = lookups * ALU_OPS_PER_4BIT_WEIGHT / (t_ms / 1e3)
         alu_peak = torch.cuda.get_device_properties(device).multi_processor_count * INT_LANES_PER_SM * mhz * 1e6

@@ -81,6 +81,12 @@ struct FwdArgs {
   const int* tiles;
   const int* perm;
   int64_t lut_task_stride;  // elements between consecutive LUT sets
+  // grid order: 0 = (split, row block, token tile), token tiles slowest, so the
+  // CTAs in flight share X columns and every token tile sweeps the index map
+  // (kept in L2 when it is the smaller operand); 1 = (1, token tile, row block),
+  // token tiles fastest, so the CTAs in flight share their row blocks' index
+  // rows and X (the smaller operand) stays in L2
+  int tiles_fast;
 };
 
 // The thread's CH consecutive 32-column chunks of the step, starting at chunk
@@ -129,16 +135,17 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
 
   const int warp = tc::warp_id(), lane = tc::lane_id();
   const int ks = blockIdx.x, ksplit = gridDim.x;
-  const int64_t m0 = (int64_t)blockIdx.y * 128;
-  int t0 = blockIdx.z * N;       // first X row of the tile
+  const int mb = a.tiles_fast ? blockIdx.z : blockIdx.y, tt = a.tiles_fast ? blockIdx.y : blockIdx.z;
+  const int64_t m0 = (int64_t)mb * 128;
+  int t0 = tt * N;               // first X row of the tile
   int tlen = N;                  // tokens of the tile (bounded by T below)
   const uint16_t* lut = a.lut;
   if (a.tiles != nullptr) {
     // the routing kernel wrote the tile list: wait for it before the setup
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int tau = a.tiles[3 * blockIdx.z];
-    t0 = a.tiles[3 * blockIdx.z + 1];
-    tlen = a.tiles[3 * blockIdx.z + 2];
+    const int tau = a.tiles[3 * tt];
+    t0 = a.tiles[3 * tt + 1];
+    tlen = a.tiles[3 * tt + 2];
     if (tlen == 0) return;       // the whole cluster shares the tile and leaves together
     lut += (int64_t)tau * a.lut_task_stride;
   } else if (t0 + tlen > a.T) {
@@ -394,12 +401,19 @@ cudaError_t launch_n(const Problem& p, const uint16_t* X, uint16_t* Y, cudaStrea
     const int forced = env_int("SK_TC_KSPLIT", 0);
     if (forced >= 1 && forced <= 8) ksplit = forced <= steps ? forced : 1;
   }
+  // keep the smaller of the index map and X in L2: sweep the token tiles
+  // fastest when the index map is the larger (only without a K split)
+  const int64_t idx_bytes = p.n * p.row_bytes, x_bytes = p.T * p.d * 2;
+  int tiles_fast = ksplit == 1 && t_tiles > 1 && idx_bytes > x_bytes ? 1 : 0;
+  const int forced_order = env_int("SK_TC_ORDER", -1);
+  if (ksplit == 1 && (forced_order == 0 || forced_order == 1)) tiles_fast = forced_order;
   FwdArgs args{p.lut, p.n, p.d, p.gs, p.T, p.gpr, steps, Y, p.check,
                rt != nullptr ? rt->tiles : nullptr, rt != nullptr ? rt->perm : nullptr,
-               p.n * p.gpr * (1 << BITS)};
+               p.n * p.gpr * (1 << BITS), tiles_fast};
 
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)ksplit, (unsigned)m_blocks, (unsigned)t_tiles);
+  cfg.gridDim = tiles_fast ? dim3(1u, (unsigned)t_tiles, (unsigned)m_blocks)
+                           : dim3((unsigned)ksplit, (unsigned)m_blocks, (unsigned)t_tiles);
   cfg.blockDim = dim3(C::THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = s;

@@ -38,6 +38,7 @@ def test_training_flops_are_three_products():
     ("dlut", 8192, "finetune7b_mt", "dlut_tc_kernel (routed)"),
     ("fwd", 1, "serve70b_decode", "decode_group_kernel"),
     ("fwd", 64, "serve70b_decode", "fwd_tc_kernel (routed)"),
+    ("fwd", 4096, "serve70b_prefill", "fwd_tc_kernel (routed)"),
 ])
 def test_kernel_attribution(op, T, workload, name, monkeypatch):
     monkeypatch.delenv("SK_FWD_PATH", raising=False)
