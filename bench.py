@@ -152,17 +152,27 @@ def launch_flops(n, d, T, op):
     return 2 * T * n * d  # each of Y, dX and the dense part of dLUT is one T x n x d contraction
 
 
+def fwd_tc_kernel_name(T, ntask):
+    """The tensor-core forward kernel for a batch: 256-token tiles (more than
+    128 tokens per LUT set on average) run on a CTA pair unless SK_TC_PAIR=0."""
+    per = -(-T // ntask)
+    pair = per > 128 and os.environ.get("SK_TC_PAIR", "1") != "0"
+    return "fwd_tc_pair_kernel" if pair else "fwd_tc_kernel"
+
+
 def kernel_name(op, T, w):
     """The library kernel a launch of this kind runs (the dispatch rules of sk_api.cu)."""
     if op == "fwd":
         if w["ntask"] > 1:
-            return "decode_group_kernel" if (w["bits"] == 4 and T == 1) else "fwd_tc_kernel (routed)"
+            if w["bits"] == 4 and T == 1:
+                return "decode_group_kernel"
+            return fwd_tc_kernel_name(T, w["ntask"]) + " (routed)"
         path = os.environ.get("SK_FWD_PATH", "")
         if w["bits"] == 4 and T <= 16 and path not in ("gemv", "tc"):
             return "decode_group_kernel"
         if path == "gemv" or (T == 1 and path != "tc"):
             return "gemv_fwd_single_kernel"
-        return "fwd_tc_kernel"
+        return fwd_tc_kernel_name(T, 1)
     routed = " (routed)" if w["ntask"] > 1 else ""
     if op == "dx":
         return "dx_tc_kernel" + routed if T >= 64 else "simt_bwd_input_kernel"

@@ -69,6 +69,9 @@ struct DxArgs {
   const int* tiles;
   const int* perm;
   int64_t lut_task_stride;
+  // 1: the epilogue writes whole token rows of dX from shared memory with bulk
+  // copies (16-byte aligned dX); 0: each thread stores its own column
+  int y_bulk;
 };
 
 template <int BITS>
@@ -237,8 +240,12 @@ dx_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, DxArgs a) {
     const int64_t j = j0 + quad * 32 + lane;
     bool have = !*abort_flag && tc::mbar_wait(d_full, 0, a.check);
     have = __all_sync(0xffffffffu, have);  // tcgen05.ld is warp-collective
-    if (have) {
-      tc::tc_fence_after();
+    if (have) tc::tc_fence_after();
+    if (a.y_bulk) {
+      // the stage memory is free: every MMA has completed (d_full)
+      tc::store_tile_bulk<N, 8>(reinterpret_cast<uint16_t*>(smem), tmem, have, warp, lane, j0, a.d, t0, (int)tlen,
+                                a.tiles != nullptr ? a.perm : nullptr, a.dX);
+    } else if (have) {
       for (int gi = (warp >> 2); gi < N / 16; gi += 2) {
         uint32_t v[16];
         tc::tmem_ld16(tc::tmem_addr(tmem, quad * 32, gi * 16), v);
@@ -495,9 +502,10 @@ cudaError_t dx_launch(const Problem& p, const uint16_t* dY, uint16_t* dX, const 
   cudaError_t e = make_tmap_2d(&tm, rt != nullptr ? rt->Xp : dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)p.n,
                                (uint64_t)p.T, (uint64_t)p.n * 2, 64, dx::N, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
+  const int y_bulk = p.d % 8 == 0 && (reinterpret_cast<uintptr_t>(dX) & 15) == 0 && env_int("SK_TC_YBULK", 1) != 0;
   DxArgs args{p.packed, p.row_bytes, p.lut, p.n, p.d, p.gs, p.T, p.gpr, dX, p.check,
               rt != nullptr ? rt->tiles : nullptr, rt != nullptr ? rt->perm : nullptr,
-              p.n * p.gpr * (1 << p.bits)};
+              p.n * p.gpr * (1 << p.bits), y_bulk ? 1 : 0};
   dim3 grid((unsigned)ceil_div(p.d, 128), rt != nullptr ? (unsigned)rt->max_tiles : (unsigned)ceil_div(p.T, dx::N));
   auto run = [&](auto kern) {
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dx::SMEM);

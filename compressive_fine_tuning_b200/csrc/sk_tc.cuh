@@ -113,6 +113,27 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// Bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned)
+// from this CTA's shared memory to global memory, in the current bulk group.
+// Shared-memory writes of the generic proxy must be fenced (fence_async_smem)
+// before the copy is issued.
+__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+               ::"l"(reinterpret_cast<uint64_t>(gdst)), "r"(smem_u32(ssrc)), "r"(bytes) : "memory");
+}
+
+// close the current bulk group and wait until every bulk copy this thread
+// issued has finished reading shared memory (the global writes complete
+// with the grid)
+__device__ __forceinline__ void bulk_commit_wait_read() {
+  asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// named barrier over the first `threads` threads of the CTA (a multiple of 32)
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // ----------------------------------------------------------------------------
 // tensor memory
 // ----------------------------------------------------------------------------
@@ -238,6 +259,130 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                : "memory");
+}
+
+
+// Epilogue of a 128 x N output tile held in tensor memory (TMEM lane = output
+// column of Y or dX, i.e. a weight row or a weight column; TMEM column =
+// token): the first DQW warps read the fp32 accumulator,
+// round it to bf16 into `ys` ([N tokens][128], token-major, in free stage
+// memory), then every token row goes to its output row (out row = perm[t0 + t]
+// for task-routed tiles, else t0 + t) with one bulk copy of min(128, n - m0)
+// values; `n` is the output row length.  Needs n % 8 == 0 and a 16-byte
+// aligned output.  Warp w reads lanes 32 (w % 4) .. + 31
+// and token groups w / 4, w / 4 + DQW / 4, ...; `have` false writes zeros.
+template <int N, int DQW>
+__device__ __forceinline__ void store_tile_bulk(uint16_t* ys, uint32_t tmem_acc, bool have, int warp, int lane,
+                                                int64_t m0, int64_t n, int t0, int tlen, const int* perm,
+                                                uint16_t* Y) {
+  constexpr int PARTS = DQW / 4;
+  const int quad = warp & 3, part = warp >> 2;
+  const int r = quad * 32 + lane;
+  for (int gi = part; gi < N / 16; gi += PARTS) {
+    uint32_t v[16];
+    if (have) {
+      tmem_ld16(tmem_addr(tmem_acc, quad * 32, gi * 16), v);
+      tmem_ld_wait();
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = 0u;
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(v[j]));
+      ys[(gi * 16 + j) * 128 + r] = *reinterpret_cast<uint16_t*>(&b);
+    }
+  }
+  fence_async_smem();
+  named_bar_sync(1, DQW * 32);
+  const int64_t rows = n - m0 < 128 ? n - m0 : 128;
+  if (rows > 0) {
+    for (int t = threadIdx.x; t < tlen; t += DQW * 32) {
+      const int64_t orow = perm != nullptr ? (int64_t)perm[t0 + t] : (int64_t)(t0 + t);
+      bulk_store(Y + orow * n + m0, ys + t * 128, (uint32_t)(rows * 2));
+    }
+    bulk_commit_wait_read();
+  }
+}
+
+// ----------------------------------------------------------------------------
+// CTA pairs (cluster of two, cta_group::2): the even CTA of the pair issues
+// the MMAs for both, each CTA supplies half of every operand tile from its own
+// shared and tensor memory, and the accumulator rows are split between the two
+// tensor memories.  Barriers that the MMA thread waits on live in the even CTA.
+// ----------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// shared::cluster address of the same shared-memory location in CTA `rank`
+__device__ __forceinline__ uint32_t mapa(const void* p, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+  return a;
+}
+
+// arrive once on a barrier given by its shared::cluster address (own or peer
+// CTA).  Default (CTA-scope release) semantics: what the arrival publishes is
+// tensor-memory data, ordered by tcgen05.wait::st and
+// tcgen05.fence::before_thread_sync before it, and a cluster-scope release
+// would add a full memory fence to every pipeline step.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
+}
+
+// every thread of both CTAs of the cluster
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// 2-D tile load into this CTA's shared memory whose completion is counted on
+// a barrier of either CTA of the pair (`bar_cluster_addr`, from mapa).  No
+// multicast: each CTA loads only its own half.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster_addr, int x,
+                                                 int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(x), "r"(y)
+      : "memory");
+}
+
+// tensor memory of both CTAs at the same address; issued by the same warp of
+// each CTA of the pair
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst, uint32_t cols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(cols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t base, uint32_t cols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(base), "r"(cols) : "memory");
+}
+
+// D (+)= A * B^T over the pair: M = 256 rows, rows 0..127 of A and D in the
+// even CTA's tensor memory and 128..255 in the odd CTA's; B's first N/2 rows
+// in the even CTA's shared memory, the rest at the same offset in the odd one
+__device__ __forceinline__ void mma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// arrive once on `bar` (same offset) in both CTAs of the pair when the pair
+// MMAs issued so far complete
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}"
+      ::"r"(smem_u32(bar)) : "memory");
 }
 
 }  // namespace tc

@@ -33,16 +33,25 @@ def test_training_flops_are_three_products():
 @pytest.mark.parametrize("op,T,workload,name", [
     ("fwd", 1, "decode7b", "decode_group_kernel"),
     ("fwd", 16, "decode7b", "decode_group_kernel"),
-    ("fwd", 8192, "finetune7b", "fwd_tc_kernel"),
+    ("fwd", 8192, "finetune7b", "fwd_tc_pair_kernel"),
+    ("fwd", 128, "finetune7b", "fwd_tc_kernel"),
     ("dx", 8192, "finetune7b", "dx_tc_kernel"),
     ("dlut", 8192, "finetune7b_mt", "dlut_tc_kernel (routed)"),
     ("fwd", 1, "serve70b_decode", "decode_group_kernel"),
     ("fwd", 64, "serve70b_decode", "fwd_tc_kernel (routed)"),
-    ("fwd", 4096, "serve70b_prefill", "fwd_tc_kernel (routed)"),
+    ("fwd", 4096, "serve70b_prefill", "fwd_tc_pair_kernel (routed)"),
 ])
 def test_kernel_attribution(op, T, workload, name, monkeypatch):
     monkeypatch.delenv("SK_FWD_PATH", raising=False)
+    monkeypatch.delenv("SK_TC_PAIR", raising=False)
     assert bench.kernel_name(op, T, W[workload]) == name
+
+
+def test_kernel_attribution_single_cta_forward(monkeypatch):
+    monkeypatch.delenv("SK_FWD_PATH", raising=False)
+    monkeypatch.setenv("SK_TC_PAIR", "0")
+    assert bench.kernel_name("fwd", 8192, W["finetune7b"]) == "fwd_tc_kernel"
+    assert bench.kernel_name("fwd", 4096, W["serve70b_prefill"]) == "fwd_tc_kernel (routed)"
 
 
 def test_sketch_factor_launch_count():

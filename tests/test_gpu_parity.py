@@ -318,6 +318,78 @@ def test_identity_exact_tc_path(fwd_path, T):
 
 
 # ---------------------------------------------------------------------------
+# 256-token tiles: on a CTA pair (cta_group::2, the default) and on one CTA
+# (SK_TC_PAIR=0).  Ragged cases: the pair's second CTA with some or none of
+# its rows inside n, a tile whose second half of tokens is empty or past T,
+# K steps that end inside a group.
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("pair", ["1", "0"])
+@pytest.mark.parametrize("shape", [(256, 512, 4, 1), (136, 320, 2, 5), (264, 1376, 3, 1), (1024, 4096, 4, 8),
+                                   (520, 2752, 2, 2), (104, 640, 4, 2)])
+@pytest.mark.parametrize("T", [129, 256, 300, 513])
+def test_forward_256_token_tiles(monkeypatch, pair, shape, T):
+    sk = _sk()
+    monkeypatch.setenv("SK_FWD_PATH", "tc")
+    monkeypatch.setenv("SK_TC_PAIR", pair)
+    c = _case(shape, T, 9300 + T)
+    packed, lut, X, dY, task = gc.dev_case(c)
+    Y = sk.linear_fwd(packed, lut, c.bits, X, task)
+    gc.check_fwd(c, Y)
+    assert sk.device_check() == 0
+
+
+@pytest.mark.parametrize("pair", ["1", "0"])
+@pytest.mark.parametrize("T,ntask,shape", [(300, 3, (264, 1376, 2, 1)), (2048, 3, (512, 2048, 4, 4)),
+                                           (1500, 2, (136, 640, 3, 2))])
+def test_multitask_forward_256_token_tiles(monkeypatch, pair, T, ntask, shape):
+    sk = _sk()
+    monkeypatch.setenv("SK_TC_PAIR", pair)
+    n, d, bits, gpr = shape
+    c = synth.layer_case(9400 + T, n=n, d=d, bits=bits, gpr=gpr, T=T, ntask=ntask)
+    packed, lut, X, dY, task = gc.dev_case(c)
+    gc.check_fwd(c, sk.linear_fwd(packed, lut, c.bits, X, task))
+    assert sk.device_check() == 0
+
+
+@pytest.mark.parametrize("pair", ["1", "0"])
+@pytest.mark.parametrize("T,ntask,shape", [(300, 1, (264, 1376, 3, 1)), (64, 1, (1024, 4096, 4, 8)),
+                                           (2048, 3, (512, 2048, 4, 4)), (96, 8, (136, 512, 3, 2))])
+def test_forward_direct_store_epilogue(monkeypatch, pair, T, ntask, shape):
+    """The per-thread store epilogue (SK_TC_YBULK=0; the library's choice when
+    Y is not 16-byte aligned) on the tensor-core forward."""
+    sk = _sk()
+    monkeypatch.setenv("SK_FWD_PATH", "tc")
+    monkeypatch.setenv("SK_TC_PAIR", pair)
+    monkeypatch.setenv("SK_TC_YBULK", "0")
+    n, d, bits, gpr = shape
+    c = synth.layer_case(9450 + T, n=n, d=d, bits=bits, gpr=gpr, T=T, ntask=ntask)
+    packed, lut, X, dY, task = gc.dev_case(c)
+    gc.check_fwd(c, sk.linear_fwd(packed, lut, c.bits, X, task))
+    assert sk.device_check() == 0
+
+
+@pytest.mark.parametrize("T", [300, 512])
+def test_identity_exact_pair_path(monkeypatch, T):
+    """Identity weights through the CTA pair: Y equals X bit for bit, so every
+    row of both CTAs and every token of both X halves lands in its place."""
+    sk = _sk()
+    monkeypatch.setenv("SK_FWD_PATH", "tc")
+    monkeypatch.setenv("SK_TC_PAIR", "1")
+    n = 1024
+    rng = synth.rng_for(9500 + T)
+    idx = torch.eye(n, dtype=torch.uint8, device="cuda")
+    packed = sk.pack(idx, 2)
+    lut = torch.full((1, n, 1, 4), float("nan"), dtype=torch.float16, device="cuda")
+    lut[..., 0] = 0.0
+    lut[..., 1] = 1.0
+    X = torch.from_numpy(synth.make_bf16(rng, (T, n), 1.0).view(np.int16)).cuda().view(torch.bfloat16)
+    Y = sk.linear_fwd(packed, lut, 2, X)
+    assert torch.equal(Y.view(torch.int16), X.view(torch.int16))
+    assert sk.device_check() == 0
+
+
+# ---------------------------------------------------------------------------
 # both backward kernels (SK_BWD_PATH forces one of them)
 # ---------------------------------------------------------------------------
 
@@ -336,6 +408,23 @@ def test_backward_each_path(monkeypatch, path, shape, T):
     gc.check_bwd_input(c, sk.linear_bwd_input(packed, lut, c.bits, c.d, dY, task))
     dl = sk.linear_bwd_lut(packed, c.bits, c.gpr, X, dY, task, 1)
     gc.check_dlut(dl.cpu().numpy()[0], oracle.backward_lut(c.x, c.dy, c.idx, c.gpr, c.k))
+    assert sk.device_check() == 0
+
+
+@pytest.mark.parametrize("ybulk", ["1", "0"])
+@pytest.mark.parametrize("T,ntask,shape", [(300, 1, (264, 1376, 3, 1)), (513, 1, (1024, 4096, 2, 8)),
+                                           (200, 3, (136, 512, 3, 2)), (700, 8, (128, 2752, 4, 2))])
+def test_bwd_input_tc_both_epilogues(monkeypatch, ybulk, T, ntask, shape):
+    """The tensor-core input gradient with its shared-memory bulk-copy
+    epilogue (the default) and with per-thread stores (SK_TC_YBULK=0), single
+    and task-routed."""
+    sk = _sk()
+    monkeypatch.setenv("SK_BWD_PATH", "tc")
+    monkeypatch.setenv("SK_TC_YBULK", ybulk)
+    n, d, bits, gpr = shape
+    c = synth.layer_case(9550 + T, n=n, d=d, bits=bits, gpr=gpr, T=T, ntask=ntask)
+    packed, lut, X, dY, task = gc.dev_case(c)
+    gc.check_bwd_input(c, sk.linear_bwd_input(packed, lut, c.bits, c.d, dY, task))
     assert sk.device_check() == 0
 
 
