@@ -369,6 +369,20 @@ def test_forward_direct_store_epilogue(monkeypatch, pair, T, ntask, shape):
     assert sk.device_check() == 0
 
 
+@pytest.mark.parametrize("T,ntask,shape", [(8000, 1, (2048, 512, 2, 2)), (9000, 1, (520, 1376, 3, 1)),
+                                           (6000, 3, (1024, 1024, 4, 4))])
+def test_forward_pair_many_tiles(monkeypatch, T, ntask, shape):
+    """Many 256 x 256 tiles (more than one wave of CTA pairs), ragged T, and
+    task-routed tiles of three sets."""
+    sk = _sk()
+    monkeypatch.setenv("SK_TC_PAIR", "1")
+    n, d, bits, gpr = shape
+    c = synth.layer_case(9480 + T, n=n, d=d, bits=bits, gpr=gpr, T=T, ntask=ntask)
+    packed, lut, X, dY, task = gc.dev_case(c)
+    gc.check_fwd(c, sk.linear_fwd(packed, lut, c.bits, X, task))
+    assert sk.device_check() == 0
+
+
 @pytest.mark.parametrize("T", [300, 512])
 def test_identity_exact_pair_path(monkeypatch, T):
     """Identity weights through the CTA pair: Y equals X bit for bit, so every
