@@ -175,7 +175,10 @@ def kernel_name(op, T, w):
         return fwd_tc_kernel_name(T, 1)
     routed = " (routed)" if w["ntask"] > 1 else ""
     if op == "dx":
-        return "dx_tc_kernel" + routed if T >= 64 else "simt_bwd_input_kernel"
+        if T < 64:
+            return "simt_bwd_input_kernel"
+        # 256-column blocks on CTA pairs unless SK_DX_PAIR=0
+        return ("dx_tc_pair_kernel" if os.environ.get("SK_DX_PAIR", "1") != "0" else "dx_tc_kernel") + routed
     return "dlut_tc_kernel" + routed if T >= 64 else "simt_bwd_lut_kernel"
 
 

@@ -55,6 +55,25 @@ constexpr uint32_t IDESC = tc::idesc_bf16(128, N, /*a MN-major*/ 1, /*b K-major*
 constexpr int TMEM_COLS = 256;
 }  // namespace dx
 
+// dX on CTA pairs (cta_group::2): the two CTAs of a cluster own 128 columns
+// each of a 256-column block and share one 256-token tile.  Each dequantises
+// its own columns' A tile into its own shared memory and loads only half of
+// the dY tile (128 tokens); the even CTA issues M = 256, N = 256 MMAs.  Half
+// the dY bytes per CTA and step let three stages fit beside two CTAs per SM.
+namespace dxp {
+constexpr int N = 256;                       // tokens per pair tile
+constexpr int KS = dx::KS;
+constexpr int S = 3;
+constexpr int B_BYTES = (N / 2) * 128;       // this CTA's 128 dY rows x 64 bf16
+constexpr int A_BYTES = dx::A_BYTES;
+constexpr int STAGE = B_BYTES + A_BYTES;
+constexpr int BAR_OFF = S * STAGE;
+constexpr int SMEM = 1024 + BAR_OFF + 256;
+constexpr uint32_t IDESC = tc::idesc_bf16(256, N, /*a MN-major*/ 1, /*b K-major*/ 0);
+constexpr int TMEM_COLS = 256;
+static_assert(N * 128 * 2 <= BAR_OFF, "the epilogue stages the output tile in the stage memory");
+}  // namespace dxp
+
 struct DxArgs {
   const uint8_t* packed;
   int64_t row_bytes;
@@ -73,6 +92,91 @@ struct DxArgs {
   // copies (16-byte aligned dX); 0: each thread stores its own column
   int y_bulk;
 };
+
+// The dequantising producers of dX (both dX kernels): warp w (of 8) fills
+// K-group w (8 rows) of every step's 128-column x 64-row A tile (MN-major,
+// 128-byte swizzle); lane = (chunk h, row r8).  wait_slot(i) waits until step
+// i's A slot may be overwritten, slot(i) is its shared-memory base and
+// ready(i) tells the MMA issuer that it is written.
+template <int BITS, class WaitSlot, class Slot, class Ready>
+__device__ __forceinline__ void dx_produce_a(const DxArgs& a, const uint16_t* lut, int64_t j0, int nsteps, int warp,
+                                             int lane, volatile int* abort_flag, WaitSlot wait_slot, Slot slot,
+                                             Ready ready) {
+  using dx::KS;
+  const int r8 = lane & 7, h = lane >> 3;
+  const int lr = 8 * warp + r8;                    // row within the step
+  const int64_t j = j0 + 32 * h;                   // first column of this thread's chunk
+  const bool col_ok = j < a.d;
+  const int64_t cchunk = j >> 5;
+  const int64_t g = col_ok ? j / a.gs : 0;
+  const int m_atom = h >> 1;
+  // swizzled 16-byte slots of this thread's four chunks within the K-row
+  uint32_t slot_off[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) slot_off[q] = m_atom * 8192 + warp * 1024 + r8 * 128 + (((4 * (h & 1) + q) ^ r8) << 4);
+  // software pipeline: this step's index chunk and raw LUT entries are loaded one step ahead
+  Chunk<BITS> ch_next{};
+  uint4 lraw_next[2] = {};
+  auto fetch = [&](int i) {
+    const int64_t row = (int64_t)i * KS + lr;
+    if (col_ok && row < a.n) {
+      ch_next = load_chunk<BITS>(a.packed + row * a.row_bytes, cchunk);
+      const uint16_t* lp = lut + (row * a.gpr + g) * (1 << BITS);
+      if constexpr (BITS == 4) {
+        lraw_next[0] = __ldg(reinterpret_cast<const uint4*>(lp));
+        lraw_next[1] = __ldg(reinterpret_cast<const uint4*>(lp) + 1);
+      } else if constexpr (BITS == 3) {
+        lraw_next[0] = __ldg(reinterpret_cast<const uint4*>(lp));
+      } else {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(lp));
+        lraw_next[0] = make_uint4(v.x, v.y, 0u, 0u);
+      }
+    }
+  };
+  fetch(0);
+  for (int i = 0; i < nsteps; ++i) {
+    const Chunk<BITS> ch = ch_next;
+    const uint4 l0 = lraw_next[0], l1 = lraw_next[1];
+    const bool ok = col_ok && (int64_t)i * KS + lr < a.n;
+    if (i + 1 < nsteps) fetch(i + 1);
+    uint32_t o[16];
+    if (ok) {
+      LutRegs<BITS> L;
+      if constexpr (BITS == 4) {
+        uint32_t w[8] = {h2_to_bf2(l0.x), h2_to_bf2(l0.y), h2_to_bf2(l0.z), h2_to_bf2(l0.w),
+                         h2_to_bf2(l1.x), h2_to_bf2(l1.y), h2_to_bf2(l1.z), h2_to_bf2(l1.w)};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          L.lo[q] = prmt(w[2 * q], w[2 * q + 1], 0x6420);
+          L.hi[q] = prmt(w[2 * q], w[2 * q + 1], 0x7531);
+        }
+      } else if constexpr (BITS == 3) {
+        uint32_t w[4] = {h2_to_bf2(l0.x), h2_to_bf2(l0.y), h2_to_bf2(l0.z), h2_to_bf2(l0.w)};
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          L.lo[q] = prmt(w[2 * q], w[2 * q + 1], 0x6420);
+          L.hi[q] = prmt(w[2 * q], w[2 * q + 1], 0x7531);
+        }
+      } else {
+        const uint32_t w0 = h2_to_bf2(l0.x), w1 = h2_to_bf2(l0.y);
+        L.lo[0] = prmt(w0, w1, 0x6420);
+        L.hi[0] = prmt(w0, w1, 0x7531);
+      }
+      dequant_chunk<BITS>(ch, L, o);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) o[e] = 0u;
+    }
+    if (*abort_flag || !wait_slot(i)) { *abort_flag = 1; break; }
+    uint8_t* at = slot(i);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      *reinterpret_cast<uint4*>(at + slot_off[q]) = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+    tc::fence_async_smem();
+    __syncwarp();
+    if (lane == 0) ready(i);
+  }
+}
 
 template <int BITS>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -156,81 +260,11 @@ dx_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, DxArgs a) {
       if (ok) tc::mma_commit(d_full);
     }
   } else {
-    // producers: warp w fills K-group w (8 rows) of the A tile; lane = (chunk h, row r8)
-    const int r8 = lane & 7, h = lane >> 3;
-    const int lr = 8 * warp + r8;                    // row within the step
-    const int64_t j = j0 + 32 * h;                   // first column of this thread's chunk
-    const bool col_ok = j < a.d;
-    const int64_t cchunk = j >> 5;
-    const int64_t g = col_ok ? j / a.gs : 0;
-    const int m_atom = h >> 1;
-    // swizzled 16-byte slots of this thread's four chunks within the K-row
-    uint32_t slot_off[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) slot_off[q] = m_atom * 8192 + warp * 1024 + r8 * 128 + (((4 * (h & 1) + q) ^ r8) << 4);
-    // software pipeline: this step's index chunk and raw LUT entries are loaded one step ahead
-    Chunk<BITS> ch_next{};
-    uint4 lraw_next[2] = {};
-    auto fetch = [&](int i) {
-      const int64_t row = (int64_t)i * KS + lr;
-      if (col_ok && row < a.n) {
-        ch_next = load_chunk<BITS>(a.packed + row * a.row_bytes, cchunk);
-        const uint16_t* lp = lut + (row * a.gpr + g) * (1 << BITS);
-        if constexpr (BITS == 4) {
-          lraw_next[0] = __ldg(reinterpret_cast<const uint4*>(lp));
-          lraw_next[1] = __ldg(reinterpret_cast<const uint4*>(lp) + 1);
-        } else if constexpr (BITS == 3) {
-          lraw_next[0] = __ldg(reinterpret_cast<const uint4*>(lp));
-        } else {
-          const uint2 v = __ldg(reinterpret_cast<const uint2*>(lp));
-          lraw_next[0] = make_uint4(v.x, v.y, 0u, 0u);
-        }
-      }
-    };
-    fetch(0);
-    for (int i = 0; i < nsteps; ++i) {
-      const int s = i % S;
-      const Chunk<BITS> ch = ch_next;
-      const uint4 l0 = lraw_next[0], l1 = lraw_next[1];
-      const bool ok = col_ok && (int64_t)i * KS + lr < a.n;
-      if (i + 1 < nsteps) fetch(i + 1);
-      uint32_t o[16];
-      if (ok) {
-        LutRegs<BITS> L;
-        if constexpr (BITS == 4) {
-          uint32_t w[8] = {h2_to_bf2(l0.x), h2_to_bf2(l0.y), h2_to_bf2(l0.z), h2_to_bf2(l0.w),
-                           h2_to_bf2(l1.x), h2_to_bf2(l1.y), h2_to_bf2(l1.z), h2_to_bf2(l1.w)};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            L.lo[q] = prmt(w[2 * q], w[2 * q + 1], 0x6420);
-            L.hi[q] = prmt(w[2 * q], w[2 * q + 1], 0x7531);
-          }
-        } else if constexpr (BITS == 3) {
-          uint32_t w[4] = {h2_to_bf2(l0.x), h2_to_bf2(l0.y), h2_to_bf2(l0.z), h2_to_bf2(l0.w)};
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            L.lo[q] = prmt(w[2 * q], w[2 * q + 1], 0x6420);
-            L.hi[q] = prmt(w[2 * q], w[2 * q + 1], 0x7531);
-          }
-        } else {
-          const uint32_t w0 = h2_to_bf2(l0.x), w1 = h2_to_bf2(l0.y);
-          L.lo[0] = prmt(w0, w1, 0x6420);
-          L.hi[0] = prmt(w0, w1, 0x7531);
-        }
-        dequant_chunk<BITS>(ch, L, o);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) o[e] = 0u;
-      }
-      if (*abort_flag || !tc::mbar_wait(&empty[s], ((i / S) & 1) ^ 1, a.check)) { *abort_flag = 1; break; }
-      uint8_t* at = smem + s * STAGE + B_BYTES;
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<uint4*>(at + slot_off[q]) = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-      tc::fence_async_smem();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&full_a[s]);
-    }
+    // producers: dequantise Θ̂ᵀ into this step's A slot
+    dx_produce_a<BITS>(a, lut, j0, nsteps, warp, lane, abort_flag,
+                       [&](int i) { return tc::mbar_wait(&empty[i % S], ((i / S) & 1) ^ 1, a.check); },
+                       [&](int i) { return smem + (i % S) * STAGE + B_BYTES; },
+                       [&](int i) { tc::mbar_arrive(&full_a[i % S]); });
   }
 
   // epilogue: thread = column j (TMEM lane), warps w and w + 4 split the tokens
@@ -268,6 +302,142 @@ dx_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, DxArgs a) {
   if (warp == kMmaWarp) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(kThreads, 2)
+dx_tc_pair_kernel(const __grid_constant__ CUtensorMap tm_dy, DxArgs a) {
+  using namespace dxp;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full_b = reinterpret_cast<uint64_t*>(smem + BAR_OFF);  // even CTA: both dY halves landed
+  uint64_t* full_a = full_b + S;                                    // even CTA: both A tiles written
+  uint64_t* empty = full_a + S;                                     // both CTAs: the pair MMAs read the stage
+  uint64_t* d_full = empty + S;                                     // both CTAs: accumulator final
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(d_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = tc::warp_id(), lane = tc::lane_id();
+  const uint32_t rank = tc::cluster_ctarank();                      // 0: issues the MMAs
+  const int64_t j0 = (int64_t)(blockIdx.x >> 1) * 256 + 128 * rank;
+  int t0 = blockIdx.y * N;
+  int64_t tlen = a.T - t0;
+  const uint16_t* lut = a.lut;
+  if (a.tiles != nullptr) {
+    const int tau = a.tiles[3 * blockIdx.y];
+    t0 = a.tiles[3 * blockIdx.y + 1];
+    tlen = a.tiles[3 * blockIdx.y + 2];
+    if (tlen == 0) return;            // both CTAs of the pair read the same entry and leave together
+    lut += (int64_t)tau * a.lut_task_stride;
+  }
+  if (tlen > N) tlen = N;
+  auto out_row = [&](int t) -> int64_t { return a.tiles != nullptr ? (int64_t)a.perm[t0 + t] : (int64_t)(t0 + t); };
+  const int nsteps = ceil_div(a.n, KS);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      tc::mbar_init(&full_b[s], 1);
+      tc::mbar_init(&full_a[s], 16);
+      tc::mbar_init(&empty[s], 1);
+    }
+    tc::mbar_init(d_full, 1);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == kMmaWarp) tc::tmem_alloc_pair(tmem_slot, TMEM_COLS);
+  if (warp == kTmaWarp && lane == 0) tc::tma_prefetch(&tm_dy);
+  tc::tc_fence_before();
+  // both CTAs' barriers are initialised before either CTA signals the other
+  tc::cluster_sync_all();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kTmaWarp) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < nsteps && !*abort_flag; ++i) {
+        const int s = i % S;
+        if (!tc::mbar_wait(&empty[s], ((i / S) & 1) ^ 1, a.check)) { *abort_flag = 1; break; }
+        // the even CTA's full_b counts the dY bytes of both CTAs
+        if (rank == 0) tc::mbar_arrive_expect_tx(&full_b[s], 2 * B_BYTES);
+        tc::tma_load_2d_pair(smem + s * STAGE, &tm_dy, tc::mapa(&full_b[s], 0), i * KS, t0 + 128 * (int)rank);
+        ++issued;
+      }
+      // never leave with a copy still landing in shared memory: the pair MMAs
+      // read every landed half before they free its stage
+      bool ok = true;
+      for (int k = issued > S ? issued - S : 0; k < issued && ok; ++k)
+        ok = tc::mbar_wait(&empty[k % S], (k / S) & 1, a.check);
+    }
+  } else if (warp == kMmaWarp) {
+    if (rank == 0 && lane == 0) {
+      bool ok = true;
+      for (int i = 0; i < nsteps; ++i) {
+        const int s = i % S;
+        if (*abort_flag || !tc::mbar_wait(&full_b[s], (i / S) & 1, a.check) ||
+            !tc::mbar_wait(&full_a[s], (i / S) & 1, a.check)) {
+          *abort_flag = 1; ok = false; break;
+        }
+        tc::tc_fence_after();
+        const uint32_t bb = tc::smem_u32(smem + s * STAGE);
+        const uint32_t ab = bb + B_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < KS / 16; ++kk) {
+          const uint64_t ad = tc::sdesc(ab + kk * 2048, 8192, 1024, tc::kSwizzle128);
+          const uint64_t bd = tc::sdesc(bb + kk * 32, 16, 1024, tc::kSwizzle128);
+          tc::mma_ss_pair(tmem, ad, bd, IDESC, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc::mma_commit_pair(&empty[s]);
+      }
+      if (ok) tc::mma_commit_pair(d_full);
+    }
+  } else {
+    // producers: dequantise this CTA's 128 columns of Θ̂ᵀ; the even CTA's full_a counts both CTAs' warps
+    const uint32_t full_a_even = tc::mapa(&full_a[0], 0);
+    dx_produce_a<BITS>(a, lut, j0, nsteps, warp, lane, abort_flag,
+                       [&](int i) { return tc::mbar_wait(&empty[i % S], ((i / S) & 1) ^ 1, a.check); },
+                       [&](int i) { return smem + (i % S) * STAGE + B_BYTES; },
+                       [&](int i) { tc::mbar_arrive_cluster(full_a_even + 8 * (i % S)); });
+  }
+
+  // epilogue: each CTA writes its own 128 columns of dX for the pair's tokens
+  __syncthreads();
+  if (warp < 8) {
+    const int quad = warp & 3;
+    const int64_t j = j0 + quad * 32 + lane;
+    bool have = !*abort_flag && tc::mbar_wait(d_full, 0, a.check);
+    have = __all_sync(0xffffffffu, have);  // tcgen05.ld is warp-collective
+    if (have) tc::tc_fence_after();
+    if (a.y_bulk) {
+      tc::store_tile_bulk<N, 8>(reinterpret_cast<uint16_t*>(smem), tmem, have, warp, lane, j0, a.d, t0, (int)tlen,
+                                a.tiles != nullptr ? a.perm : nullptr, a.dX);
+    } else if (have) {
+      for (int gi = (warp >> 2); gi < N / 16; gi += 2) {
+        uint32_t v[16];
+        tc::tmem_ld16(tc::tmem_addr(tmem, quad * 32, gi * 16), v);
+        tc::tmem_ld_wait();
+        if (j < a.d) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int t = gi * 16 + e;
+            if (t < tlen) {
+              __nv_bfloat16 bv = __float2bfloat16_rn(__uint_as_float(v[e]));
+              a.dX[out_row(t) * a.d + j] = *reinterpret_cast<uint16_t*>(&bv);
+            }
+          }
+        }
+      }
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  // neither CTA leaves (or frees tensor memory) while the other may still
+  // signal its barriers or the pair MMAs may still use its memory
+  tc::cluster_sync_all();
+  if (warp == kMmaWarp) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc_pair(tmem, TMEM_COLS);
   }
 }
 
@@ -506,7 +676,39 @@ cudaError_t dx_launch(const Problem& p, const uint16_t* dY, uint16_t* dX, const 
   DxArgs args{p.packed, p.row_bytes, p.lut, p.n, p.d, p.gs, p.T, p.gpr, dX, p.check,
               rt != nullptr ? rt->tiles : nullptr, rt != nullptr ? rt->perm : nullptr,
               p.n * p.gpr * (1 << p.bits), y_bulk ? 1 : 0};
-  dim3 grid((unsigned)ceil_div(p.d, 128), rt != nullptr ? (unsigned)rt->max_tiles : (unsigned)ceil_div(p.T, dx::N));
+  const unsigned tiles = rt != nullptr ? (unsigned)rt->max_tiles : (unsigned)ceil_div(p.T, dx::N);
+  if (env_int("SK_DX_PAIR", 1) != 0) {
+    // CTA pairs over 256-column blocks (SK_DX_PAIR=0: one CTA per 128 columns)
+    CUtensorMap tmp;
+    e = make_tmap_2d(&tmp, rt != nullptr ? rt->Xp : dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)p.n,
+                     (uint64_t)p.T, (uint64_t)p.n * 2, 64, dxp::N / 2, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
+    auto run_pair = [&](auto kern) {
+      cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dxp::SMEM);
+      if (err != cudaSuccess) return err;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2u * (unsigned)ceil_div(p.d, 256), tiles, 1u);
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = dxp::SMEM;
+      cfg.stream = s;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      err = cudaLaunchKernelEx(&cfg, kern, tmp, args);
+      if (err != cudaSuccess) return err;
+      return cudaGetLastError();
+    };
+    switch (p.bits) {
+      case 2: return run_pair(dx_tc_pair_kernel<2>);
+      case 3: return run_pair(dx_tc_pair_kernel<3>);
+      default: return run_pair(dx_tc_pair_kernel<4>);
+    }
+  }
+  dim3 grid((unsigned)ceil_div(p.d, 128), tiles);
   auto run = [&](auto kern) {
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dx::SMEM);
     if (err != cudaSuccess) return err;

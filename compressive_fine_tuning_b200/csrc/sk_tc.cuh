@@ -340,8 +340,8 @@ __device__ __forceinline__ void cluster_sync_all() {
 }
 
 // 2-D tile load into this CTA's shared memory whose completion is counted on
-// a barrier of either CTA of the pair (`bar_cluster_addr`, from mapa).  No
-// multicast: each CTA loads only its own half.
+// a barrier of either CTA of the pair (`bar_cluster_addr`, from mapa).  Each
+// CTA loads only its own half into its own shared memory.
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster_addr, int x,
                                                  int y) {
   asm volatile(
@@ -373,6 +373,19 @@ __device__ __forceinline__ void mma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, ui
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
       ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D (+)= A * B^T over the pair with both operands in shared memory: A's rows
+// 0..127 in the even CTA, 128..255 at the same offset in the odd one; B as in
+// mma_ts_pair
+__device__ __forceinline__ void mma_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 

@@ -442,6 +442,25 @@ def test_bwd_input_tc_both_epilogues(monkeypatch, ybulk, T, ntask, shape):
     assert sk.device_check() == 0
 
 
+@pytest.mark.parametrize("pair", ["1", "0"])
+@pytest.mark.parametrize("T,ntask,shape", [(64, 1, (136, 320, 2, 5)), (300, 1, (264, 1376, 3, 1)),
+                                           (513, 1, (1024, 4096, 2, 8)), (700, 8, (128, 2752, 4, 2)),
+                                           (1000, 3, (520, 640, 4, 4))])
+def test_bwd_input_pair_and_single(monkeypatch, pair, T, ntask, shape):
+    """The tensor-core input gradient on CTA pairs (two 128-column halves of a
+    256-column block, the default) and on one CTA per 128 columns
+    (SK_DX_PAIR=0): ragged columns (a pair whose second half is past d) and
+    tokens, single and task-routed."""
+    sk = _sk()
+    monkeypatch.setenv("SK_BWD_PATH", "tc")
+    monkeypatch.setenv("SK_DX_PAIR", pair)
+    n, d, bits, gpr = shape
+    c = synth.layer_case(9700 + T, n=n, d=d, bits=bits, gpr=gpr, T=T, ntask=ntask)
+    packed, lut, X, dY, task = gc.dev_case(c)
+    gc.check_bwd_input(c, sk.linear_bwd_input(packed, lut, c.bits, c.d, dY, task))
+    assert sk.device_check() == 0
+
+
 def test_bwd_lut_tc_workspace_required():
     sk = _sk()
     c = _case((256, 512, 4, 1), 128, 9600)
