@@ -27,9 +27,22 @@ constexpr int kMaxDevices = 64;
 std::atomic<int> g_sms[kMaxDevices];
 }  // namespace
 
+// The tensor-map encoder is a driver call and needs a context current on the
+// calling thread.  A thread that has made no runtime call yet (an autograd
+// worker thread, a plain host thread of the caller) has none, so bind the
+// current device's primary context once per thread, as the first runtime call
+// of a launch would.
+static void bind_context() {
+  thread_local bool bound = false;
+  if (bound) return;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && cudaSetDevice(dev) == cudaSuccess) bound = true;
+}
+
 cudaError_t make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem_bytes,
                          uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
                          uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+  bind_context();
   std::call_once(g_encode_once, load_encode);
   if (g_encode_err != cudaSuccess) return g_encode_err;
   (void)elem_bytes;
@@ -46,6 +59,7 @@ cudaError_t make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType
 cudaError_t make_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, uint64_t dim0,
                          uint64_t dim1, uint64_t dim2, uint64_t stride1, uint64_t stride2, uint32_t box0,
                          uint32_t box1, uint32_t box2, CUtensorMapSwizzle swizzle) {
+  bind_context();
   std::call_once(g_encode_once, load_encode);
   if (g_encode_err != cudaSuccess) return g_encode_err;
   cuuint64_t dims[3] = {dim0, dim1, dim2};

@@ -247,6 +247,36 @@ def test_autograd_function():
     gc.check_dlut(L2.grad.float().cpu().numpy()[0], ref, "lut.grad")
 
 
+def test_entry_points_from_a_fresh_thread():
+    """Every tensor-core entry point called from a host thread that has made no
+    CUDA call yet (as an autograd worker thread may be): the library binds the
+    device's context before its first driver call (the tensor-map encoder)."""
+    import threading
+    sk = _sk()
+    c = _case((264, 1376, 3, 1), 300, 7400)
+    packed, lut, X, dY, task = gc.dev_case(c)
+    torch.cuda.synchronize()
+    out, err = {}, []
+
+    def run():
+        try:
+            out["Y"] = sk.linear_fwd(packed, lut, c.bits, X)
+            out["dX"] = sk.linear_bwd_input(packed, lut, c.bits, c.d, dY)
+            out["dl"] = sk.linear_bwd_lut(packed, c.bits, c.gpr, X, dY)
+            torch.cuda.synchronize()
+        except Exception as e:  # reported in the test's own thread
+            err.append(e)
+
+    t = threading.Thread(target=run)
+    t.start()
+    t.join()
+    assert not err, err
+    gc.check_fwd(c, out["Y"])
+    gc.check_bwd_input(c, out["dX"])
+    gc.check_dlut(out["dl"].cpu().numpy()[0], oracle.backward_lut(c.x, c.dy, c.idx, c.gpr, c.k))
+    assert sk.device_check() == 0
+
+
 def test_autograd_function_fp32_master_lut():
     """An fp32 master LUT gets the library's fp32 LUT gradient unrounded
     (1024 tokens, dY ~ N(0, 1e-2), the 2e-3 bounds)."""
@@ -458,6 +488,27 @@ def test_bwd_input_pair_and_single(monkeypatch, pair, T, ntask, shape):
     c = synth.layer_case(9700 + T, n=n, d=d, bits=bits, gpr=gpr, T=T, ntask=ntask)
     packed, lut, X, dY, task = gc.dev_case(c)
     gc.check_bwd_input(c, sk.linear_bwd_input(packed, lut, c.bits, c.d, dY, task))
+    assert sk.device_check() == 0
+
+
+@pytest.mark.parametrize("pair", ["1", "0"])
+@pytest.mark.parametrize("T,ntask,shape", [(64, 1, (136, 320, 2, 5)), (300, 1, (264, 1376, 3, 1)),
+                                           (513, 1, (1024, 4096, 2, 8)), (700, 8, (128, 2752, 4, 2)),
+                                           (1000, 3, (520, 640, 4, 4))])
+def test_bwd_lut_pair_and_single(monkeypatch, pair, T, ntask, shape):
+    """The tensor-core LUT gradient on CTA pairs (two 128-row halves of a
+    256-row block, the default) and on one CTA per 128 rows (SK_DLUT_PAIR=0):
+    ragged rows (a pair whose second half is past n) and tokens, single and
+    task-routed."""
+    sk = _sk()
+    monkeypatch.setenv("SK_BWD_PATH", "tc")
+    monkeypatch.setenv("SK_DLUT_PAIR", pair)
+    n, d, bits, gpr = shape
+    c = synth.layer_case(9750 + T, n=n, d=d, bits=bits, gpr=gpr, T=T, ntask=ntask)
+    packed, lut, X, dY, task = gc.dev_case(c)
+    dl = sk.linear_bwd_lut(packed, c.bits, c.gpr, X, dY, task, ntask)
+    ref = oracle.backward_lut(c.x, c.dy, c.idx, c.gpr, c.k, task=c.task, ntask=ntask)
+    gc.check_dlut(dl.cpu().numpy().reshape(ref.shape), ref)
     assert sk.device_check() == 0
 
 
