@@ -179,7 +179,10 @@ def kernel_name(op, T, w):
             return "simt_bwd_input_kernel"
         # 256-column blocks on CTA pairs unless SK_DX_PAIR=0
         return ("dx_tc_pair_kernel" if os.environ.get("SK_DX_PAIR", "1") != "0" else "dx_tc_kernel") + routed
-    return "dlut_tc_kernel" + routed if T >= 64 else "simt_bwd_lut_kernel"
+    if T < 64:
+        return "simt_bwd_lut_kernel"
+    # 256-row blocks on CTA pairs unless SK_DLUT_PAIR=0
+    return ("dlut_tc_pair_kernel" if os.environ.get("SK_DLUT_PAIR", "1") != "0" else "dlut_tc_kernel") + routed
 
 
 def kernels_per_launch(op, T, w):

@@ -464,6 +464,25 @@ constexpr uint32_t IDESC = tc::idesc_bf16(M, N, 1, 1);
 constexpr int TMEM_COLS = 256;
 }  // namespace dl
 
+// The LUT gradient on CTA pairs (cta_group::2): the two CTAs of a cluster own
+// 128 rows each of a 256-row block and share one 256-column tile; each loads
+// its own dY rows and half of the X tile (128 columns), the even CTA issues
+// M = 256, N = 256 MMAs, and each CTA bins its own rows' accumulator as
+// above.  Half the X bytes per CTA and step let three stages fit beside two
+// CTAs per SM.
+namespace dlp {
+constexpr int N = 256;
+constexpr int KS = dl::KS;
+constexpr int A_BYTES = dl::A_BYTES;        // this CTA's 128 rows of dY^T
+constexpr int B_BYTES = 2 * 8192;           // this CTA's 128 columns of X
+constexpr int STAGE = A_BYTES + B_BYTES;
+constexpr int S = 3;
+constexpr int BAR_OFF = S * STAGE;
+constexpr int SMEM = 1024 + BAR_OFF + 256;
+constexpr uint32_t IDESC = tc::idesc_bf16(256, N, 1, 1);
+constexpr int TMEM_COLS = 256;
+}  // namespace dlp
+
 // Group slots of one 256-column tile: groups [tile*256 / gs, (tile*256 + 255) / gs].
 __host__ __device__ inline int dlut_slots(int64_t gs, int gpr) {
   const int64_t s = 255 / gs + 2;
@@ -482,6 +501,7 @@ struct DlutArgs {
   // nullptr for one LUT set
   const int* segs;
   int64_t part_task_stride;  // floats between the partial bins of consecutive LUT sets
+  int row_pairs;             // CTA-pair kernel: 256-row blocks per LUT set
 };
 
 template <int BITS>
@@ -630,6 +650,166 @@ dlut_tc_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant_
   }
 }
 
+template <int BITS>
+__global__ void __launch_bounds__(dl::THREADS, 2)
+dlut_tc_pair_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_x, DlutArgs a) {
+  using namespace dlp;
+  constexpr int K = 1 << BITS, TMA_WARP = dl::TMA_WARP, MMA_WARP = dl::MMA_WARP;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + BAR_OFF);   // even CTA: both CTAs' operands landed
+  uint64_t* empty = full + S;                                      // both CTAs: the pair MMAs read the stage
+  uint64_t* d_full = empty + S;                                    // both CTAs: accumulator final
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(d_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = tc::warp_id(), lane = tc::lane_id();
+  const uint32_t rank = tc::cluster_ctarank();                     // 0: issues the MMAs
+  // grid: (pair, column tile, row block + row_pairs * LUT set), column tiles
+  // fastest after the pair, so the clusters in flight cover all column tiles
+  // of a few row blocks
+  const int jt = blockIdx.y;
+  const int64_t j0 = (int64_t)jt * N;
+  const int set = (int)blockIdx.z / a.row_pairs;
+  const int64_t i0 = (int64_t)((int)blockIdx.z - set * a.row_pairs) * 256 + 128 * rank;
+  int k_first = 0;
+  int nsteps = ceil_div(a.T, KS);
+  float* part = a.part;
+  if (a.segs != nullptr) {
+    k_first = a.segs[2 * set];
+    nsteps = ceil_div(a.segs[2 * set + 1], KS);   // a set with no tokens writes zero partials
+    part += (int64_t)set * a.part_task_stride;
+  }
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    tc::mbar_init(d_full, 1);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == MMA_WARP) tc::tmem_alloc_pair(tmem_slot, TMEM_COLS);
+  if (warp == TMA_WARP && lane == 0) {
+    tc::tma_prefetch(&tm_dy);
+    tc::tma_prefetch(&tm_x);
+  }
+  tc::tc_fence_before();
+  // both CTAs' barriers are initialised before either CTA signals the other
+  tc::cluster_sync_all();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == TMA_WARP) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < nsteps && !*abort_flag; ++i) {
+        const int s = i % S;
+        if (!tc::mbar_wait(&empty[s], ((i / S) & 1) ^ 1, a.check)) { *abort_flag = 1; break; }
+        uint8_t* st = smem + s * STAGE;
+        // the even CTA's full counts the operand bytes of both CTAs
+        if (rank == 0) tc::mbar_arrive_expect_tx(&full[s], 2 * STAGE);
+        const uint32_t bar = tc::mapa(&full[s], 0);
+        const int tk = k_first + i * KS;
+        tc::tma_load_2d_pair(st, &tm_dy, bar, (int)i0, tk);
+        tc::tma_load_2d_pair(st + 8192, &tm_dy, bar, (int)i0 + 64, tk);
+        const int jx = (int)j0 + 128 * (int)rank;
+        tc::tma_load_2d_pair(st + A_BYTES, &tm_x, bar, jx, tk);
+        tc::tma_load_2d_pair(st + A_BYTES + 8192, &tm_x, bar, jx + 64, tk);
+        ++issued;
+      }
+      // never leave with a copy still landing in shared memory: the pair MMAs
+      // read every landed stage before they free it
+      bool ok = true;
+      for (int k = issued > S ? issued - S : 0; k < issued && ok; ++k)
+        ok = tc::mbar_wait(&empty[k % S], (k / S) & 1, a.check);
+    }
+  } else if (warp == MMA_WARP) {
+    if (rank == 0 && lane == 0) {
+      bool ok = true;
+      for (int i = 0; i < nsteps; ++i) {
+        const int s = i % S;
+        if (*abort_flag || !tc::mbar_wait(&full[s], (i / S) & 1, a.check)) { *abort_flag = 1; ok = false; break; }
+        tc::tc_fence_after();
+        const uint32_t ab = tc::smem_u32(smem + s * STAGE), bb = ab + A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < KS / 16; ++kk) {
+          const uint64_t ad = tc::sdesc(ab + kk * 2048, 8192, 1024, tc::kSwizzle128);
+          const uint64_t bd = tc::sdesc(bb + kk * 2048, 8192, 1024, tc::kSwizzle128);
+          tc::mma_ss_pair(tmem, ad, bd, IDESC, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc::mma_commit_pair(&empty[s]);
+      }
+      if (ok) tc::mma_commit_pair(d_full);
+    }
+  } else {
+    // epilogue warps 0-3: thread = row i (TMEM lane); bin the row's 256 columns
+    float* bins = reinterpret_cast<float*>(smem + BAR_OFF - K * 128 * 4);  // [K][128], tail of stage memory
+    const int tid = threadIdx.x;                                         // 0..127
+    const int64_t i = i0 + tid;
+    Chunk<BITS> chunks[N / 32];
+#pragma unroll
+    for (int q = 0; q < N / 32; ++q) {
+      const int64_t jc = j0 + 32 * q;
+      if (i < a.n && jc < a.d) chunks[q] = load_chunk<BITS>(a.packed + i * a.row_bytes, jc >> 5);
+    }
+    bool have = !*abort_flag && tc::mbar_wait(d_full, 0, a.check) && nsteps > 0;   // no steps: nothing accumulated
+    have = __all_sync(0xffffffffu, have);  // tcgen05.ld is warp-collective
+    if (have) tc::tc_fence_after();
+    // the bins reuse the last stage's memory: every MMA has read it (d_full)
+#pragma unroll
+    for (int c = 0; c < K; ++c) bins[c * 128 + tid] = 0.f;
+    const int first_g = (int)(j0 / a.gs);
+    const int gs32 = (int)a.gs;
+    int g = first_g, g_end = (first_g + 1) * gs32;
+    bool dirty = false;
+    auto flush = [&](int gg) {
+      if (i < a.n) {
+        float* dst = part + (((int64_t)jt * a.n + i) * a.slots + (gg - first_g)) * K;
+#pragma unroll
+        for (int c = 0; c < K; ++c) dst[c] = bins[c * 128 + tid];
+      }
+#pragma unroll
+      for (int c = 0; c < K; ++c) bins[c * 128 + tid] = 0.f;
+    };
+#pragma unroll
+    for (int q = 0; q < N / 32; ++q) {
+      const int64_t jc = j0 + 32 * q;
+      if (jc >= a.d) break;
+      uint32_t v[32];
+      if (have) {
+        tc::tmem_ld32(tc::tmem_addr(tmem, warp * 32, 32 * q), v);
+        tc::tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = 0u;
+      }
+      if ((int)jc >= g_end) {
+        if (dirty) flush(g);
+        do { ++g; g_end += gs32; } while ((int)jc >= g_end);
+        dirty = false;
+      }
+      if (i < a.n) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) bins[chunk_index<BITS>(chunks[q], e) * 128 + tid] += __uint_as_float(v[e]);
+      }
+      dirty = true;
+    }
+    if (dirty) flush(g);
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  // neither CTA leaves (or frees tensor memory) while the other may still
+  // signal its barriers or the pair MMAs may still use its memory
+  tc::cluster_sync_all();
+  if (warp == MMA_WARP) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+}
+
 // Sum the partial bins of every (row, group) over the column tiles that touch
 // the group, in tile order, and write (or add to) dlut.
 template <int BITS>
@@ -753,23 +933,45 @@ cudaError_t dlut_launch(const Problem& p, const uint16_t* X, const uint16_t* dY,
   const int sets = rp != nullptr ? p.ntask : 1;
   const int64_t stride = (int64_t)jtiles * p.n * slots * (1 << p.bits);
   DlutArgs args{p.packed, p.row_bytes, p.n, p.d, p.gs, p.T, p.gpr, slots, part, p.check,
-                rp != nullptr ? rp->segs : nullptr, stride};
-  dim3 grid((unsigned)jtiles, (unsigned)ceil_div(p.n, dl::M), (unsigned)sets);
+                rp != nullptr ? rp->segs : nullptr, stride, ceil_div(p.n, 256)};
   const int64_t outs = (int64_t)sets * p.n * p.gpr * (1 << p.bits);
   const unsigned rgrid = (unsigned)((outs + 255) / 256);
-  auto run = [&](auto kern, auto red) {
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dl::SMEM);
+  // 256-row blocks on CTA pairs unless SK_DLUT_PAIR=0
+  const bool pair = env_int("SK_DLUT_PAIR", 1) != 0;
+  auto run = [&](auto kern, auto kern_pair, auto red) {
+    cudaError_t err;
+    if (pair) {
+      err = cudaFuncSetAttribute(kern_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, dlp::SMEM);
+      if (err != cudaSuccess) return err;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2u, (unsigned)jtiles, (unsigned)(ceil_div(p.n, 256) * sets));
+      cfg.blockDim = dim3(dl::THREADS, 1, 1);
+      cfg.dynamicSmemBytes = dlp::SMEM;
+      cfg.stream = s;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      err = cudaLaunchKernelEx(&cfg, kern_pair, tm_dy, tm_x, args);
+    } else {
+      err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dl::SMEM);
+      if (err != cudaSuccess) return err;
+      dim3 grid((unsigned)jtiles, (unsigned)ceil_div(p.n, dl::M), (unsigned)sets);
+      kern<<<grid, dl::THREADS, dl::SMEM, s>>>(tm_dy, tm_x, args);
+    }
     if (err != cudaSuccess) return err;
-    kern<<<grid, dl::THREADS, dl::SMEM, s>>>(tm_dy, tm_x, args);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     red<<<rgrid, 256, 0, s>>>(part, p.n, p.gpr, p.gs, jtiles, slots, dlut, accumulate, sets, stride);
     return cudaGetLastError();
   };
   switch (p.bits) {
-    case 2: return run(dlut_tc_kernel<2>, dlut_reduce_kernel<2>);
-    case 3: return run(dlut_tc_kernel<3>, dlut_reduce_kernel<3>);
-    default: return run(dlut_tc_kernel<4>, dlut_reduce_kernel<4>);
+    case 2: return run(dlut_tc_kernel<2>, dlut_tc_pair_kernel<2>, dlut_reduce_kernel<2>);
+    case 3: return run(dlut_tc_kernel<3>, dlut_tc_pair_kernel<3>, dlut_reduce_kernel<3>);
+    default: return run(dlut_tc_kernel<4>, dlut_tc_pair_kernel<4>, dlut_reduce_kernel<4>);
   }
 }
 }  // namespace

@@ -37,7 +37,7 @@ def test_training_flops_are_three_products():
     ("fwd", 128, "finetune7b", "fwd_tc_kernel"),
     ("dx", 8192, "finetune7b", "dx_tc_pair_kernel"),
     ("dx", 8192, "finetune7b_mt", "dx_tc_pair_kernel (routed)"),
-    ("dlut", 8192, "finetune7b_mt", "dlut_tc_kernel (routed)"),
+    ("dlut", 8192, "finetune7b_mt", "dlut_tc_pair_kernel (routed)"),
     ("fwd", 1, "serve70b_decode", "decode_group_kernel"),
     ("fwd", 64, "serve70b_decode", "fwd_tc_kernel (routed)"),
     ("fwd", 4096, "serve70b_prefill", "fwd_tc_pair_kernel (routed)"),
@@ -46,6 +46,7 @@ def test_kernel_attribution(op, T, workload, name, monkeypatch):
     monkeypatch.delenv("SK_FWD_PATH", raising=False)
     monkeypatch.delenv("SK_TC_PAIR", raising=False)
     monkeypatch.delenv("SK_DX_PAIR", raising=False)
+    monkeypatch.delenv("SK_DLUT_PAIR", raising=False)
     assert bench.kernel_name(op, T, W[workload]) == name
 
 
@@ -56,6 +57,8 @@ def test_kernel_attribution_single_cta_forward(monkeypatch):
     assert bench.kernel_name("fwd", 4096, W["serve70b_prefill"]) == "fwd_tc_kernel (routed)"
     monkeypatch.setenv("SK_DX_PAIR", "0")
     assert bench.kernel_name("dx", 8192, W["finetune7b"]) == "dx_tc_kernel"
+    monkeypatch.setenv("SK_DLUT_PAIR", "0")
+    assert bench.kernel_name("dlut", 8192, W["finetune7b"]) == "dlut_tc_kernel"
 
 
 def test_sketch_factor_launch_count():
