@@ -51,6 +51,11 @@
  *
  * Streams: every call is asynchronous on the given stream (NULL = the legacy
  * default stream).
+ *
+ * Devices and threads: a call runs on the calling thread's current CUDA device
+ * (cudaSetDevice).  Any host thread may call, including one that has made no
+ * CUDA call yet (an autograd worker thread, for instance): the library binds
+ * that device's primary context to the thread before its first driver call.
  */
 #ifndef SK_H_
 #define SK_H_
