@@ -66,8 +66,9 @@ def test_decode_forward_7b_shapes(monkeypatch, n, d, T):
 
 @pytest.mark.parametrize("T", [1, 16])
 def test_decode_matches_tensor_core_path_and_is_deterministic(monkeypatch, T):
-    """Both kernels round the same bf16 weights; fp32 sums in different orders
-    agree to a few bf16 ulps, and the decode kernel repeats itself bit for bit."""
+    """Each kernel meets the oracle on every element; the two (the same bf16
+    weights, fp32 sums in different orders) agree to a few bf16 ulps, and the
+    decode kernel repeats itself bit for bit."""
     from compressive_fine_tuning_b200 import sk
     c = synth.layer_case(33000 + T, n=4096, d=4096, bits=4, gpr=8, T=T)
     packed, lut, X, dY, task = gc.dev_case(c)
@@ -77,6 +78,8 @@ def test_decode_matches_tensor_core_path_and_is_deterministic(monkeypatch, T):
     assert torch.equal(y1, y2)
     monkeypatch.setenv("SK_FWD_PATH", "tc")
     y3 = sk.linear_fwd(packed, lut, 4, X, task)
+    gc.check_fwd(c, y1)
+    gc.check_fwd(c, y3)
     a, b = y1.float(), y3.float()
     assert torch.allclose(a, b, rtol=2 ** -6, atol=1e-3 * b.abs().max().item())
 
